@@ -1,0 +1,335 @@
+/*
+ * fp6_oracle.c -- plain, slow CPU reference for the FP6 (e3m2) weight-only
+ * linear layer.  TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the
+ * benchmark's CPU-baseline leg are the only callers.  The CUDA library never
+ * links, includes or calls this file, and this file shares no code, header or
+ * table with it.
+ *
+ * Sources (web pages on the method):
+ *   - "FP6-LLM: Efficiently Serving Large Language Models Through FP6-Centric
+ *     Algorithm-System Co-Design", abstract: weights quantized to 6-bit floats,
+ *     activations stay FP16 (W6A16).
+ *   - duicuo.cn news article on TC-FPx, section "kernel solution redesign":
+ *     dequantization turns FP6 into FP16 before the tensor-core product; weights
+ *     are pre-packed offline and each 6-bit weight is split into a 2-bit and a
+ *     4-bit piece stored in aligned 32-bit words.
+ * The pages fix neither the bit format nor the scale; the format used here is
+ * e3m2 with exponent bias 3, no inf/NaN, maximum magnitude 28, and one FP16
+ * scale per output row (the layer's stated specification).
+ *
+ * Every floating-point step is done in IEEE binary64 unless stated.
+ *
+ * Parity status of each function (what pins it, all in tests/):
+ *   decode table        pinned: closed form over all 64 codes + golden file
+ *   f16 rounding        pinned: numpy float16 conversion (library routine)
+ *   quantize            pinned: exact brute-force argmin, round trip, error
+ *                       bound, CUDA's own fp6 conversion routine
+ *   prepack / unpack    pinned: bit-splice decode of the packed words gives the
+ *                       closed-form fp16 pattern; one-hot probe; round trip
+ *   dequant             pinned: closed form of decode*scale rounded by numpy
+ *   linear              pinned: exact rational dot products (tiny shapes),
+ *                       one-hot and constant-code special cases
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <pthread.h>
+
+#define ORC_OK 0
+#define ORC_ERR_INVALID_ARG 1
+#define ORC_ERR_UNSUPPORTED_SHAPE 2
+#define ORC_ERR_NONFINITE 4
+#define ORC_ERR_SCALE_RANGE 5
+
+/* ------------------------------------------------------------------------ */
+/* FP16 <-> binary64                                                         */
+/* ------------------------------------------------------------------------ */
+
+/* Value of an IEEE binary16 bit pattern, exactly. */
+double oracle_f16_to_f64(uint16_t h)
+{
+    int sign = (h >> 15) & 1;
+    int e = (h >> 10) & 0x1F;
+    int f = h & 0x3FF;
+    double v;
+    if (e == 0) {
+        v = ldexp((double)f, -24);               /* subnormal: f * 2^-24 */
+    } else if (e == 31) {
+        v = f ? NAN : INFINITY;
+    } else {
+        v = ldexp((double)(1024 + f), e - 25);   /* (1 + f/1024) * 2^(e-15) */
+    }
+    return sign ? -v : v;
+}
+
+/* Round a binary64 value to the nearest binary16, ties to even.
+ * Magnitudes at or above 65520 (the midpoint past 65504) become infinity. */
+uint16_t oracle_f64_to_f16_rne(double v)
+{
+    uint16_t sign = signbit(v) ? 0x8000u : 0u;
+    double a = fabs(v);
+    if (isnan(v)) return 0x7E00u;
+    if (isinf(a)) return sign | 0x7C00u;
+    if (a == 0.0) return sign;
+    if (a < ldexp(1.0, -14)) {
+        /* subnormal range: count in units of 2^-24 (exact scaling) */
+        double q = nearbyint(ldexp(a, 24));
+        return sign | (uint16_t)q;   /* q == 1024 is the smallest normal */
+    }
+    int ex;
+    frexp(a, &ex);          /* a = f * 2^ex with f in [0.5, 1) */
+    int e = ex - 1;         /* a in [2^e, 2^(e+1)) */
+    double q = nearbyint(ldexp(a, 10 - e));      /* in [1024, 2048] */
+    int biased = e + 15;
+    if (biased >= 31) return sign | 0x7C00u;
+    uint32_t bits = ((uint32_t)biased << 10) + ((uint32_t)q - 1024u);
+    if (bits >= 0x7C00u) return sign | 0x7C00u; /* rounded past 65504 */
+    return sign | (uint16_t)bits;
+}
+
+/* ------------------------------------------------------------------------ */
+/* FP6 e3m2 decode (table-driven)                                            */
+/* ------------------------------------------------------------------------ */
+
+/* Code bits, low 6 bits of a byte: b5 = sign, b4..b2 = exponent e, b1..b0 =
+ * mantissa m.  e > 0: (-1)^s * 2^(e-3) * (1 + m/4);  e == 0: (-1)^s * 2^-2 * m/4. */
+static double g_decode[64];
+static int g_decode_ready = 0;
+
+static void build_decode_table(void)
+{
+    for (int c = 0; c < 64; ++c) {
+        int s = (c >> 5) & 1, e = (c >> 2) & 7, m = c & 3;
+        double mag = (e > 0) ? ldexp(1.0 + m / 4.0, e - 3) : ldexp(m / 4.0, -2);
+        g_decode[c] = s ? -mag : mag;
+    }
+    g_decode_ready = 1;
+}
+
+static inline double decode(uint8_t c)
+{
+    return g_decode[c & 0x3F];
+}
+
+void oracle_decode_table(double *out64)
+{
+    if (!g_decode_ready) build_decode_table();
+    for (int c = 0; c < 64; ++c) out64[c] = g_decode[c];
+}
+
+/* Round v to the nearest e3m2 value, ties to the even mantissa, saturating to
+ * +-28 (there is no infinity code).  The sign bit of v is kept, so negative
+ * values that round to zero give the code 0x20.  Steps: find the binade of
+ * |v| (or the subnormal range), scale |v| to units of that binade's spacing,
+ * round to an integer with ties to even, and rebuild the code; a carry out of
+ * the mantissa lands on the next binade's first code. */
+uint8_t oracle_round_e3m2(double v)
+{
+    uint8_t sign = signbit(v) ? 0x20u : 0u;
+    double a = fabs(v);
+    int code;
+    if (a < 0.25) {
+        /* subnormal spacing 2^-4; the quotient 4 is the code of 0.25 */
+        code = (int)nearbyint(ldexp(a, 4));
+    } else {
+        int ex;
+        frexp(a, &ex);
+        int e = ex - 1;                       /* a in [2^e, 2^(e+1)) */
+        if (e > 4) {
+            code = 32;                        /* beyond the top binade */
+        } else {
+            double q = nearbyint(ldexp(a, 2 - e));   /* in [4, 8] */
+            code = ((e + 3) << 2) + ((int)q - 4);
+        }
+    }
+    if (code > 31) code = 31;                 /* saturate at 28 */
+    return sign | (uint8_t)code;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Quantize: one fp16 scale per output row, then RNE e3m2 codes              */
+/* ------------------------------------------------------------------------ */
+
+/* Per row n:  amax = max_k |W[n,k]|;  s = fp16_rne(fp32(amax / 28));
+ * code[n,k] = round_e3m2(W[n,k] / s)  (binary64 division, correctly rounded).
+ * A row of zeros gets s = 0 and codes 0.  Any non-finite weight is an error;
+ * a scale that overflows or underflows fp16 is an error. */
+int oracle_quantize(const float *W, int64_t N, int64_t K, uint8_t *codes, uint16_t *scales)
+{
+    if (N < 0 || K < 0) return ORC_ERR_INVALID_ARG;
+    if (!g_decode_ready) build_decode_table();
+    for (int64_t n = 0; n < N; ++n) {
+        const float *row = W + n * K;
+        float amax = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            if (!isfinite(row[k])) return ORC_ERR_NONFINITE;
+            float a = fabsf(row[k]);
+            if (a > amax) amax = a;
+        }
+        if (amax == 0.0f) {
+            scales[n] = 0;
+            memset(codes + n * K, 0, (size_t)K);
+            continue;
+        }
+        volatile float s32 = amax / 28.0f;                 /* IEEE fp32 division */
+        uint16_t s16 = oracle_f64_to_f16_rne((double)s32);
+        if ((s16 & 0x7FFFu) >= 0x7C00u || (s16 & 0x7FFFu) == 0) return ORC_ERR_SCALE_RANGE;
+        scales[n] = s16;
+        double s = oracle_f16_to_f64(s16);
+        for (int64_t k = 0; k < K; ++k) {
+            double v = (double)row[k] / s;
+            codes[n * K + k] = oracle_round_e3m2(v);
+        }
+    }
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Prepack / unpack: 2+4 bit split into 32-bit-aligned fragment streams      */
+/* ------------------------------------------------------------------------ */
+
+/* Packed layout (version 1).  W is cut into tiles of 128 rows x 64 columns,
+ * stored tile after tile with the column-tile index fastest:
+ *     tile (nt, kt) at byte (nt * (K/64) + kt) * 6144.
+ * Inside a tile, row r (0..127) owns twelve 32-bit words:
+ *     lo words L_q, q = 0..7, at byte (q/4)*2048 + r*16 + (q%4)*4
+ *     hi words H_p, p = 0..3, at byte 4096 + r*16 + p*4
+ * Column kk (0..63) of the tile belongs to pair j = kk/2, half h = kk%2.
+ * The code's low four bits (e1 e0 m1 m0) sit in L_{j/4} at bit 4*(j%4) + 16*h.
+ * The code's top two bits sit in H_{j/8}, with i = j%8:
+ *     e2 (code bit 4) at bit 2*i + 16*h,
+ *     s  (code bit 5) at bit (2*i + 3 + 16*h) mod 32.
+ * Byte order is little-endian (bit b of a word is bit b%8 of byte b/8). */
+static inline int64_t tile_base(int64_t n, int64_t k, int64_t K)
+{
+    return ((n / 128) * (K / 64) + (k / 64)) * 6144;
+}
+
+static inline void put_bit(uint8_t *buf, int64_t word_byte, int bit, int value)
+{
+    if (value) buf[word_byte + bit / 8] |= (uint8_t)(1u << (bit % 8));
+}
+
+static inline int get_bit(const uint8_t *buf, int64_t word_byte, int bit)
+{
+    return (buf[word_byte + bit / 8] >> (bit % 8)) & 1;
+}
+
+int oracle_prepack(const uint8_t *codes, int64_t N, int64_t K, uint8_t *packed)
+{
+    if (N < 0 || K < 0) return ORC_ERR_INVALID_ARG;
+    if (N % 128 || K % 64) return ORC_ERR_UNSUPPORTED_SHAPE;
+    memset(packed, 0, (size_t)(N * K / 4 * 3));
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < K; ++k) {
+            uint8_t c = codes[n * K + k] & 0x3F;
+            int64_t base = tile_base(n, k, K);
+            int r = (int)(n % 128), kk = (int)(k % 64);
+            int j = kk / 2, h = kk % 2;
+            int q = j / 4, p = j / 8, i = j % 8;
+            int64_t lo_word = base + (q / 4) * 2048 + r * 16 + (q % 4) * 4;
+            int64_t hi_word = base + 4096 + r * 16 + p * 4;
+            int lo_bit = 4 * (j % 4) + 16 * h;
+            for (int b = 0; b < 4; ++b) put_bit(packed, lo_word, lo_bit + b, (c >> b) & 1);
+            put_bit(packed, hi_word, 2 * i + 16 * h, (c >> 4) & 1);
+            put_bit(packed, hi_word, (2 * i + 3 + 16 * h) % 32, (c >> 5) & 1);
+        }
+    }
+    return ORC_OK;
+}
+
+int oracle_unpack(const uint8_t *packed, int64_t N, int64_t K, uint8_t *codes)
+{
+    if (N < 0 || K < 0) return ORC_ERR_INVALID_ARG;
+    if (N % 128 || K % 64) return ORC_ERR_UNSUPPORTED_SHAPE;
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < K; ++k) {
+            int64_t base = tile_base(n, k, K);
+            int r = (int)(n % 128), kk = (int)(k % 64);
+            int j = kk / 2, h = kk % 2;
+            int q = j / 4, p = j / 8, i = j % 8;
+            int64_t lo_word = base + (q / 4) * 2048 + r * 16 + (q % 4) * 4;
+            int64_t hi_word = base + 4096 + r * 16 + p * 4;
+            int lo_bit = 4 * (j % 4) + 16 * h;
+            uint8_t c = 0;
+            for (int b = 0; b < 4; ++b) c |= (uint8_t)(get_bit(packed, lo_word, lo_bit + b) << b);
+            c |= (uint8_t)(get_bit(packed, hi_word, 2 * i + 16 * h) << 4);
+            c |= (uint8_t)(get_bit(packed, hi_word, (2 * i + 3 + 16 * h) % 32) << 5);
+            codes[n * K + k] = c;
+        }
+    }
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Dequant: W16[n,k] = fp16(decode(c)) or fp16_rne(decode(c) * s[n])          */
+/* ------------------------------------------------------------------------ */
+
+int oracle_dequant(const uint8_t *packed, const uint16_t *scales, int64_t N, int64_t K, uint16_t *W16)
+{
+    if (N < 0 || K < 0) return ORC_ERR_INVALID_ARG;
+    if (N % 128 || K % 64) return ORC_ERR_UNSUPPORTED_SHAPE;
+    if (!g_decode_ready) build_decode_table();
+    uint8_t *codes = (uint8_t *)malloc((size_t)(N * K) + 1);
+    if (!codes) return ORC_ERR_INVALID_ARG;
+    oracle_unpack(packed, N, K, codes);
+    for (int64_t n = 0; n < N; ++n) {
+        double s = scales ? oracle_f16_to_f64(scales[n]) : 1.0;
+        for (int64_t k = 0; k < K; ++k)
+            W16[n * K + k] = oracle_f64_to_f16_rne(decode(codes[n * K + k]) * s);
+    }
+    free(codes);
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Linear: y[m,n] = fp16_rne( sum_k x[m,k] * (s[n] * decode(C[n,k])) )        */
+/* ------------------------------------------------------------------------ */
+
+/* The plain definition of the layer: weights reconstructed as s[n]*decode,
+ * multiplied with the fp16 activations; each product is exact in binary64
+ * (at most 25 significant bits) and the sum runs over k in ascending order.
+ * One rounding to fp16 at the end. */
+typedef struct {
+    const uint16_t *x; const uint8_t *codes; const uint16_t *scales;
+    int64_t M, N, K, n0, n1; uint16_t *y;
+} linear_job;
+
+static void *linear_rows(void *arg)
+{
+    linear_job *jb = (linear_job *)arg;
+    double *xr = (double *)malloc(sizeof(double) * (size_t)(jb->K > 0 ? jb->K : 1));
+    for (int64_t m = 0; m < jb->M; ++m) {
+        for (int64_t k = 0; k < jb->K; ++k) xr[k] = oracle_f16_to_f64(jb->x[m * jb->K + k]);
+        for (int64_t n = jb->n0; n < jb->n1; ++n) {
+            double s = oracle_f16_to_f64(jb->scales[n]);
+            const uint8_t *c = jb->codes + n * jb->K;
+            double acc = 0.0;
+            for (int64_t k = 0; k < jb->K; ++k) acc += xr[k] * (s * decode(c[k]));
+            jb->y[m * jb->N + n] = oracle_f64_to_f16_rne(acc);
+        }
+    }
+    free(xr);
+    return NULL;
+}
+
+int oracle_linear(const uint16_t *x, const uint8_t *codes, const uint16_t *scales,
+                  int64_t M, int64_t N, int64_t K, uint16_t *y, int nthreads)
+{
+    if (M < 0 || N < 0 || K < 0) return ORC_ERR_INVALID_ARG;
+    if (!g_decode_ready) build_decode_table();
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 256) nthreads = 256;
+    if (nthreads > N) nthreads = (int)(N > 0 ? N : 1);
+    pthread_t th[256];
+    linear_job jobs[256];
+    for (int t = 0; t < nthreads; ++t) {
+        jobs[t] = (linear_job){x, codes, scales, M, N, K,
+                               N * t / nthreads, N * (t + 1) / nthreads, y};
+    }
+    for (int t = 1; t < nthreads; ++t) pthread_create(&th[t], NULL, linear_rows, &jobs[t]);
+    linear_rows(&jobs[0]);
+    for (int t = 1; t < nthreads; ++t) pthread_join(th[t], NULL);
+    return ORC_OK;
+}
