@@ -1,0 +1,385 @@
+#!/usr/bin/env python3
+"""Benchmark of the FP6 x FP16 weight-only linear layer on B200.
+
+Workload (one "step"): the Llama-70B-shaped attention output projection,
+N = K = 8192, at decode batch sizes M = 1, 2, 4, 8, 16 -- one fp6_linear
+launch per M, each reading a different copy of the packed weights (copies
+rotate so the weights streamed per launch are never L2-resident).  Metric:
+effective weight GB/s = 0.75 * N * K bytes per launch / time.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fp6|reference]
+
+Under torchrun (N > 1) every rank runs the same independent workload on its
+own GPU (weak scaling, no data-path collective); the step time is the max over
+ranks.  `--impl reference` times the CPU oracle on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD_NAME = "llama70b_o_proj_decode"
+N_DIM, K_DIM = 8192, 8192
+MS = [1, 2, 4, 8, 16]
+METRIC = "FP6xFP16 linear: weight GB/s (M<=16) & TFLOP/s (M>=256), % of roofline"
+UNIT = "GB/s"
+
+
+def wbytes(N, K):
+    return 0.75 * N * K
+
+
+def algo_bytes(M, N, K):
+    """Algorithmic bytes of one launch: packed weights + fp16 scales + fp16 activations."""
+    return 0.75 * N * K + 2 * N + 2 * M * K
+
+
+def read_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ---- clocks sampled during the timed region ---------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, ValueError):
+            self.proc = None
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---- distributed plumbing --------------------------------------------------------
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---- the oracle (CPU baseline / reference arm) ------------------------------------
+
+def oracle_workload(rows: int):
+    """Codes/scales of the first `rows` weight rows and the activations, from the oracle."""
+    import oracle
+    from weight_only_quantized_fp6_b200 import inputs
+    wseed = inputs.weight_seed(2, 0)
+    W = inputs.weights(wseed, N_DIM, K_DIM, rows=range(rows))
+    codes, scales = oracle.quantize(W)
+    xs = {M: inputs.activations(inputs.activation_seed(wseed, M), M, K_DIM) for M in MS}
+    return codes, scales, xs
+
+
+def time_oracle(rows: int, threads: int, reps: int = 1):
+    import oracle
+    codes, scales, xs = oracle_workload(rows)
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        for M in MS:
+            oracle.linear(xs[M], codes, scales, nthreads=threads)
+    dt = time.perf_counter() - t0
+    gbs = reps * len(MS) * wbytes(rows, K_DIM) / dt / 1e9
+    return gbs, dt
+
+
+def cpu_baseline():
+    threads = os.cpu_count() or 1
+    rows = N_DIM  # the whole layer: a few seconds of all-core CPU work
+    gbs, dt = time_oracle(rows, threads)
+    return {"value": round(gbs, 4), "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"one full step (N={N_DIM}, K={K_DIM}, M={MS}) on {threads} threads, {dt:.2f} s"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    threads = os.cpu_count() or 1
+    rows = 2048  # a quarter of the layer per step keeps --steps 10 within a few minutes
+    import oracle
+    codes, scales, xs = oracle_workload(rows)
+    for _ in range(args.warmup):
+        for M in MS:
+            oracle.linear(xs[M], codes, scales, nthreads=threads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        for M in MS:
+            oracle.linear(xs[M], codes, scales, nthreads=threads)
+    dt = time.perf_counter() - t0
+    value = args.steps * len(MS) * wbytes(rows, K_DIM) / dt / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3 / args.steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": f"{WORKLOAD_NAME} N={N_DIM} K={K_DIM} M={MS}",
+                                        "rows_per_step": rows},
+        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"first {rows} of {N_DIM} weight rows, all M, per step"},
+        "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---- the GPU arm -------------------------------------------------------------------
+
+def run_fp6(args, world, rank, local):
+    import torch
+
+    import weight_only_quantized_fp6_b200 as fp6
+    from weight_only_quantized_fp6_b200 import inputs
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    props = torch.cuda.get_device_properties(dev)
+    l2 = getattr(props, "L2_cache_size", 126 * 1024 * 1024)
+
+    # weights: seeded N(0, 0.02), quantized and packed by the library
+    wseed = inputs.weight_seed(2, rank)
+    W = inputs.weights_parallel(wseed, N_DIM, K_DIM)
+    layer = fp6.FP6Linear.from_float(torch.from_numpy(W).to(dev))
+    del W
+    copies = max(2, math.ceil(4 * l2 / wbytes(N_DIM, K_DIM)))
+    packs = [layer.packed] + [layer.packed.clone() for _ in range(copies - 1)]
+    scales = layer.scales
+    xs = {M: torch.from_numpy(inputs.activations(inputs.activation_seed(wseed, M), M, K_DIM).view(np.int16))
+          .to(dev).view(torch.float16) for M in MS}
+    ys = {M: torch.empty((M, N_DIM), dtype=torch.float16, device=dev) for M in MS}
+    ws = fp6.Workspace(dev)
+    ws.get(max(fp6.workspace_bytes(M, N_DIM, K_DIM) for M in MS))
+
+    stream = torch.cuda.Stream(device=dev)
+    # One CUDA graph per rotation offset: 5 launches with timing events around each.
+    n_graphs = copies
+    graphs, ev = [], []
+    with torch.cuda.stream(stream):
+        for M in MS:  # eager warm-up (sets kernel attributes before capture)
+            fp6.linear(xs[M], packs[0], scales, N_DIM, K_DIM, out=ys[M], workspace=ws)
+        stream.synchronize()
+        for g in range(n_graphs):
+            evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2 * len(MS))]
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=stream):
+                for i, M in enumerate(MS):
+                    evs[2 * i].record()
+                    fp6.linear(xs[M], packs[(g * len(MS) + i) % copies], scales, N_DIM, K_DIM,
+                               out=ys[M], workspace=ws)
+                    evs[2 * i + 1].record()
+            graphs.append(graph)
+            ev.append(evs)
+    torch.cuda.synchronize()
+
+    def step(s):
+        graphs[s % n_graphs].replay()
+
+    with torch.cuda.stream(stream):
+        for s in range(args.warmup):
+            step(s)
+    torch.cuda.synchronize()
+    barrier(world)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    launch_ms = []
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        t_start.record()
+        for s in range(args.steps):
+            step(s)
+        t_end.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    elapsed_ms = t_start.elapsed_time(t_end)
+    # per-launch kernel durations from the events inside the last replay of each graph
+    for s in range(min(args.steps, n_graphs)):
+        evs = ev[s % n_graphs]
+        launch_ms.append([evs[2 * i].elapsed_time(evs[2 * i + 1]) for i in range(len(MS))])
+    clocks = sampler.stop()
+
+    elapsed_max = max_over_ranks(elapsed_ms, world)
+    launches = args.steps * len(MS)
+    total_bytes = world * launches * wbytes(N_DIM, K_DIM)
+    value = total_bytes / (elapsed_max / 1e3) / 1e9
+    # roofline of the dominant (only) kernel: algorithmic bytes / mean launch time
+    per_m = np.array(launch_ms).mean(axis=0) if launch_ms else np.full(len(MS), np.nan)
+    algo = np.array([algo_bytes(M, N_DIM, K_DIM) for M in MS])
+    achieved = float(algo.sum() / (per_m.sum() / 1e3) / 1e9)
+    peaks = read_peaks()
+
+    # end to end through the public API with host buffers: H2D of x, linear, D2H of y
+    x_host = {M: xs[M].cpu().pin_memory() for M in MS}
+    y_host = {M: torch.empty((M, N_DIM), dtype=torch.float16).pin_memory() for M in MS}
+    x_dev = {M: torch.empty_like(xs[M]) for M in MS}
+    h2d = sum(x_host[M].numel() * 2 for M in MS)
+    d2h = sum(y_host[M].numel() * 2 for M in MS)
+    e2e_steps = max(1, args.steps)
+
+    def e2e_step(s):
+        for i, M in enumerate(MS):
+            x_dev[M].copy_(x_host[M], non_blocking=True)
+            fp6.linear(x_dev[M], packs[(s * len(MS) + i) % copies], scales, N_DIM, K_DIM, out=ys[M],
+                       workspace=ws)
+            y_host[M].copy_(ys[M], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for s in range(args.warmup):
+            e2e_step(s)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record()
+        for s in range(e2e_steps):
+            e2e_step(s)
+        e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    e2e_value = world * e2e_steps * len(MS) * wbytes(N_DIM, K_DIM) / (e2e_ms / 1e3) / 1e9
+
+    ok = fp6.device_status(dev)
+    if ok != 0:
+        raise SystemExit(f"device error word set: {ok}")
+
+    if rank == 0:
+        cpu = cpu_baseline() if world == 1 else None
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(elapsed_max / args.steps, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f16 x e3m2 -> f32 accumulate", "data": "synthetic (seeded N(0,0.02) weights, N(0,1) fp16 x)",
+            "config": {
+                "workload": f"{WORKLOAD_NAME} N={N_DIM} K={K_DIM} M={MS}",
+                "launches_per_step": len(MS),
+                "l2": f"{copies} rotating packed-weight copies ({copies * wbytes(N_DIM, K_DIM) / 1e6:.0f} MB > 4x L2 "
+                      f"{l2 / 1e6:.0f} MB); CUDA-graph replay",
+                "per_M_us": {str(M): round(float(t) * 1e3, 3) for M, t in zip(MS, per_m)},
+                "per_M_roofline_frac": {str(M): round(algo_bytes(M, N_DIM, K_DIM) / (float(t) / 1e3) / 1e9
+                                                      / peaks["hbm_gbs"], 4) for M, t in zip(MS, per_m)},
+                "parallelism": f"independent replicas x{world}" if world > 1 else "single GPU",
+            },
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+                         "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs)",
+                         "kernel": "fp6_linear_kernel<16>"},
+            "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches,
+            "clocks": clocks,
+        }
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["fp6", "reference"], default="fp6")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            rc = run_reference(args, world, rank)
+        else:
+            rc = run_fp6(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    return rc
+
+
+if __name__ == "__main__":
+    sys.exit(main())

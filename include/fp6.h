@@ -1,0 +1,146 @@
+/*
+ * fp6.h -- C ABI of libfp6.so: FP6 (e3m2) x FP16 weight-only linear layer on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method (FP6-LLM abstract; TC-FPx article, section "kernel solution
+ * redesign"): weights are quantized offline to 6-bit floats, pre-packed into
+ * aligned 2-bit and 4-bit fragment streams, and at run time a single kernel
+ * rebuilds FP16 weights in registers and multiplies them with FP16
+ * activations on tensor cores.
+ *
+ * Format.  A code is the low 6 bits of a byte: sign (bit 5), exponent e (bits
+ * 4..2, bias 3), mantissa m (bits 1..0).  Value: (-1)^s 2^(e-3) (1 + m/4) for
+ * e > 0, (-1)^s 2^-2 (m/4) for e = 0.  No inf/NaN; largest magnitude 28.
+ * One FP16 scale per output row n:  W[n,k] ~= scale[n] * decode(code[n,k]).
+ *
+ * Conventions for every entry point.
+ *  - Pointers are DEVICE pointers owned by the caller; the library never
+ *    allocates or frees device memory.  Matrices are row-major and dense.
+ *  - Every pointer must be 16-byte aligned (else FP6_ERR_MISALIGNED).
+ *  - Shapes: N % 128 == 0 and K % 64 == 0 (else FP6_ERR_UNSUPPORTED_SHAPE);
+ *    sizes are non-negative (else FP6_ERR_INVALID_ARG).  A zero-sized problem
+ *    is a no-op that returns FP6_OK (fp6_linear with K == 0 writes y = 0).
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and runs asynchronously, except where a function says it
+ *    synchronizes.  Argument errors are returned before anything is enqueued.
+ *    A failed launch returns FP6_ERR_CUDA.
+ *  - fp16 values are passed as their 16-bit patterns (uint16_t).
+ */
+#ifndef FP6_H_
+#define FP6_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st; /* cudaStream_t is `struct CUstream_st *` */
+
+typedef enum {
+    FP6_OK = 0,
+    FP6_ERR_INVALID_ARG = 1,       /* null pointer, negative size, bad buffer size */
+    FP6_ERR_UNSUPPORTED_SHAPE = 2, /* N % 128 != 0 or K % 64 != 0, or too large */
+    FP6_ERR_MISALIGNED = 3,        /* a pointer is not 16-byte aligned */
+    FP6_ERR_NONFINITE = 4,         /* fp6_quantize met a NaN or infinite weight */
+    FP6_ERR_SCALE_RANGE = 5,       /* fp6_quantize: max|w|/28 overflows or underflows fp16 */
+    FP6_ERR_WORKSPACE = 6,         /* workspace missing or smaller than required */
+    FP6_ERR_CUDA = 8,              /* a CUDA runtime call or launch failed */
+    FP6_ERR_TIMEOUT = 9            /* a kernel's bounded wait ran out (see fp6_get_device_status) */
+} fp6_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *fp6_status_string(fp6_status status);
+
+/* Bytes of the packed weight buffer for an N x K matrix: exactly 3*N*K/4
+ * (six bits per weight, no header).  Returns 0 for unsupported shapes. */
+size_t fp6_packed_bytes(int64_t N, int64_t K);
+
+/*
+ * fp6_quantize -- offline FP6 quantization (FP6-LLM abstract: weights are
+ * quantized to 6-bit floats).  Per row n:
+ *     scale[n]  = fp16_rne( fp32( max_k |W[n,k]| / 28 ) )
+ *     code[n,k] = nearest e3m2 value to W[n,k] / scale[n], ties to even
+ *                 mantissa, saturating at +-28, sign bit copied from W
+ * A row of zeros gets scale 0 and codes 0.
+ *   W       [N,K] fp32, device, read-only
+ *   codes   [N,K] uint8, device, written (one code per byte, bits 7..6 zero)
+ *   scales  [N]   fp16 bit patterns, device, written
+ * SYNCHRONIZES the stream to report FP6_ERR_NONFINITE (a NaN/inf weight) or
+ * FP6_ERR_SCALE_RANGE (a scale that overflows or underflows fp16); on those
+ * errors the outputs are unspecified.  Any N >= 0, K >= 0 is accepted.
+ */
+fp6_status fp6_quantize(const float *W, int64_t N, int64_t K,
+                        uint8_t *codes, uint16_t *scales, struct CUstream_st *stream);
+
+/*
+ * fp6_prepack -- bit-level pre-packing (TC-FPx article: weights reorganised
+ * before inference, each 6-bit weight split into 2-bit and 4-bit pieces that
+ * are stored in aligned 32-bit words, fragments reordered so that the
+ * run-time rebuild is parallel).  Layout version 1:
+ *   tiles of 128 rows x 64 columns, tile (nt, kt) at byte (nt*(K/64)+kt)*6144;
+ *   inside a tile, row r owns 8 lo words L_q at byte (q/4)*2048 + r*16 + (q%4)*4
+ *   and 4 hi words H_p at byte 4096 + r*16 + p*4.  Tile column kk gives pair
+ *   j = kk/2, half h = kk%2; code bits 3..0 go to L_{j/4} bits 4(j%4)+16h ..+3;
+ *   code bit 4 to H_{j/8} bit 2(j%8)+16h; code bit 5 to H_{j/8} bit
+ *   (2(j%8)+3+16h) mod 32.  Words are little-endian.
+ *   codes   [N,K] uint8, device (bits 7..6 ignored)
+ *   packed  device buffer of packed_bytes >= fp6_packed_bytes(N,K), written
+ */
+fp6_status fp6_prepack(const uint8_t *codes, int64_t N, int64_t K,
+                       void *packed, size_t packed_bytes, struct CUstream_st *stream);
+
+/*
+ * fp6_dequant -- rebuild fp16 weights from packed codes (the "disguise FP6 as
+ * FP16" step of the TC-FPx article, run on its own; used for testing and for
+ * the separate dequant + GEMM comparison).
+ *   scales == NULL:  W16[n,k] = fp16(decode(code))            (exact)
+ *   scales != NULL:  W16[n,k] = fp16_rne(decode(code) * scale[n])
+ *   W16 [N,K] fp16 bit patterns, device, written
+ */
+fp6_status fp6_dequant(const void *packed, const uint16_t *scales, int64_t N, int64_t K,
+                       uint16_t *W16, struct CUstream_st *stream);
+
+/* Bytes of workspace fp6_linear needs for this problem on the current device
+ * (0 when the problem is empty).  The first 4096 bytes of a workspace hold
+ * counters that must be ZERO before its first use (cudaMemset once); every
+ * completed call leaves them zero again, whatever the problem size, so one
+ * zeroed buffer of the largest size needed serves every shape.  After a call
+ * that reported FP6_ERR_TIMEOUT, zero them again. */
+size_t fp6_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/*
+ * fp6_linear -- y[M,N] = x[M,K] . (scale (.) decode(W))^T, fp32 accumulation,
+ * fp16 output (round to nearest even).  FP6-LLM abstract (W6A16 inference);
+ * TC-FPx article (dequantization fused with the tensor-core product, software
+ * pipeline overlapping the two).
+ *   x        [M,K] fp16 bit patterns, device, read-only
+ *   packed   output of fp6_prepack for the [N,K] weight, device, read-only
+ *   scales   [N] fp16 bit patterns, device, read-only
+ *   y        [M,N] fp16 bit patterns, device, written
+ *   workspace  device buffer of at least fp6_linear_workspace_bytes(M,N,K)
+ *              bytes (zeroed once before first use, see above); may be NULL
+ *              only when that size is 0
+ * Concurrent calls must not share a workspace.  Deterministic: the same
+ * inputs give the same bits on every run.
+ */
+fp6_status fp6_linear(const uint16_t *x, const void *packed, const uint16_t *scales,
+                      int64_t M, int64_t N, int64_t K, uint16_t *y,
+                      void *workspace, size_t workspace_bytes, struct CUstream_st *stream);
+
+/* Reads and clears the device error word that kernels set when a bounded wait
+ * runs out (returns FP6_ERR_TIMEOUT then, else FP6_OK).  Synchronizes `stream`. */
+fp6_status fp6_get_device_status(struct CUstream_st *stream);
+
+/* Launch configuration fp6_linear would use (for tests and benchmarks):
+ * out[0] = MMA N-tile (tokens per tile), out[1] = pipeline stages,
+ * out[2] = persistent CTAs, out[3] = number of (token, row) tiles,
+ * out[4] = k-iterations in total.  Returns FP6_OK or an argument error. */
+fp6_status fp6_linear_plan(int64_t M, int64_t N, int64_t K, int64_t out[5]);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP6_H_ */

@@ -1,0 +1,86 @@
+"""The C-ABI library loads and exports every entry point include/fp6.h declares;
+argument validation happens on the host before any CUDA call (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from weight_only_quantized_fp6_b200 import _lib, build
+    build.build_library()
+    return _lib.load()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "fp6.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(fp6_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_binding_covers_header():
+    from weight_only_quantized_fp6_b200 import _lib
+    assert set(declared_functions()) == set(_lib.SIGNATURES)
+
+
+def test_status_strings(lib):
+    from weight_only_quantized_fp6_b200 import _lib
+    for code, name in _lib.STATUS.items():
+        assert lib.fp6_status_string(code).decode() == name
+
+
+def test_packed_bytes(lib):
+    assert lib.fp6_packed_bytes(8192, 8192) == 50331648
+    assert lib.fp6_packed_bytes(256, 512) == 98304
+    assert lib.fp6_packed_bytes(100, 64) == 0
+    assert lib.fp6_packed_bytes(128, 96) == 0
+    assert lib.fp6_packed_bytes(0, 64) == 0
+
+
+def test_host_side_validation(lib):
+    P = ctypes.c_void_p
+    ok_ptr = P(1 << 20)        # 16-byte aligned fake addresses: never dereferenced,
+    bad_ptr = P((1 << 20) + 2)  # validation fails before any launch
+    # unsupported shapes
+    assert lib.fp6_linear(ok_ptr, ok_ptr, ok_ptr, 4, 100, 64, ok_ptr, None, 0, None) == 2
+    assert lib.fp6_linear(ok_ptr, ok_ptr, ok_ptr, 4, 128, 96, ok_ptr, None, 0, None) == 2
+    assert lib.fp6_prepack(ok_ptr, 128, 100, ok_ptr, 1 << 20, None) == 2
+    assert lib.fp6_dequant(ok_ptr, None, 130, 64, ok_ptr, None) == 2
+    # negative sizes
+    assert lib.fp6_linear(ok_ptr, ok_ptr, ok_ptr, -1, 128, 64, ok_ptr, None, 0, None) == 1
+    assert lib.fp6_quantize(ok_ptr, -3, 64, ok_ptr, ok_ptr, None) == 1
+    # misaligned pointers
+    assert lib.fp6_linear(bad_ptr, ok_ptr, ok_ptr, 4, 128, 64, ok_ptr, None, 0, None) == 3
+    assert lib.fp6_linear(ok_ptr, ok_ptr, ok_ptr, 4, 128, 64, bad_ptr, None, 0, None) == 3
+    assert lib.fp6_prepack(bad_ptr, 128, 64, ok_ptr, 6144, None) == 3
+    assert lib.fp6_dequant(ok_ptr, bad_ptr, 128, 64, ok_ptr, None) == 3
+    # null pointers and short buffers
+    assert lib.fp6_linear(None, ok_ptr, ok_ptr, 4, 128, 64, ok_ptr, None, 0, None) == 1
+    assert lib.fp6_prepack(ok_ptr, 128, 64, ok_ptr, 6143, None) == 1
+    # empty problems are no-ops
+    assert lib.fp6_linear(None, None, None, 0, 128, 64, ok_ptr, None, 0, None) == 0
+    assert lib.fp6_prepack(None, 0, 64, None, 0, None) == 0
+    assert lib.fp6_quantize(None, 0, 64, None, None, None) == 0
+
+
+def test_oracle_is_not_linked_into_the_library():
+    """The product library never references the oracle."""
+    from weight_only_quantized_fp6_b200 import build
+    for f in build.SOURCES + build.HEADERS:
+        text = open(f).read()
+        assert "oracle" not in text.lower(), f
+    pkg = os.path.join(ROOT, "weight_only_quantized_fp6_b200")
+    for name in os.listdir(pkg):
+        if name.endswith(".py"):
+            assert "import oracle" not in open(os.path.join(pkg, name)).read(), name

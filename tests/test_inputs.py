@@ -25,3 +25,9 @@ def test_moments_and_outliers():
 def test_seeds_differ():
     assert not np.array_equal(inputs.weights(1, 8, 64), inputs.weights(2, 8, 64))
     assert inputs.activation_seed(inputs.weight_seed(2, 0), 16) == 2116
+
+
+def test_parallel_generation_matches():
+    a = inputs.weights(17, 300, 128, outlier_p=0.01)
+    b = inputs.weights_parallel(17, 300, 128, outlier_p=0.01, threads=7)
+    assert np.array_equal(a, b)

@@ -1,1 +1,168 @@
-"""FP6 (e3m2) x FP16 weight-only linear layer for NVIDIA B200 (sm_100a)."""
+"""FP6 (e3m2) x FP16 weight-only linear layer for NVIDIA B200 (sm_100a).
+
+Thin PyTorch-facing wrapper over libfp6.so (include/fp6.h).  PyTorch provides
+device memory and the current stream; every step of the computation runs in
+the library's CUDA kernels.
+
+    import weight_only_quantized_fp6_b200 as fp6
+    layer = fp6.FP6Linear.from_float(W)        # W: [N,K] fp32 on cuda
+    y = layer(x)                               # x: [M,K] fp16 on cuda -> [M,N] fp16
+"""
+from __future__ import annotations
+
+import ctypes
+import threading
+
+from . import _lib
+
+__all__ = ["quantize", "prepack", "dequant", "linear", "linear_plan", "workspace_bytes",
+           "packed_bytes", "device_status", "FP6Linear", "FP6Error", "Workspace"]
+
+FP6Error = _lib.FP6Error
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream(t):
+    return ctypes.c_void_p(_torch().cuda.current_stream(t.device).cuda_stream)
+
+
+def _need_cuda(name, t, dtype, dim=None):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if dim is not None and t.dim() != dim:
+        raise ValueError(f"{name} must have {dim} dimensions")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def packed_bytes(N: int, K: int) -> int:
+    return int(_lib.load().fp6_packed_bytes(N, K))
+
+
+def quantize(W):
+    """W [N,K] fp32 (cuda) -> (codes [N,K] uint8, scales [N] fp16).  Synchronizes."""
+    torch = _torch()
+    _need_cuda("W", W, torch.float32, 2)
+    N, K = W.shape
+    codes = torch.empty((N, K), dtype=torch.uint8, device=W.device)
+    scales = torch.empty((N,), dtype=torch.float16, device=W.device)
+    _lib.check(_lib.load().fp6_quantize(W.data_ptr(), N, K, codes.data_ptr(), scales.data_ptr(),
+                                        _stream(W)), "fp6_quantize")
+    return codes, scales
+
+
+def prepack(codes):
+    """codes [N,K] uint8 (cuda) -> packed uint8 buffer of 3*N*K/4 bytes."""
+    torch = _torch()
+    _need_cuda("codes", codes, torch.uint8, 2)
+    N, K = codes.shape
+    nbytes = packed_bytes(N, K)
+    if nbytes == 0 and N * K > 0:
+        raise FP6Error(2, "fp6_prepack")
+    packed = torch.empty((nbytes,), dtype=torch.uint8, device=codes.device)
+    _lib.check(_lib.load().fp6_prepack(codes.data_ptr(), N, K, packed.data_ptr(), nbytes, _stream(codes)),
+               "fp6_prepack")
+    return packed
+
+
+def dequant(packed, scales, N: int, K: int):
+    """packed -> W16 [N,K] fp16; scales None gives the unscaled e3m2 values."""
+    torch = _torch()
+    _need_cuda("packed", packed, torch.uint8, 1)
+    if scales is not None:
+        _need_cuda("scales", scales, torch.float16, 1)
+    out = torch.empty((N, K), dtype=torch.float16, device=packed.device)
+    _lib.check(_lib.load().fp6_dequant(packed.data_ptr(), scales.data_ptr() if scales is not None else None,
+                                       N, K, out.data_ptr(), _stream(packed)), "fp6_dequant")
+    return out
+
+
+def workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(_lib.load().fp6_linear_workspace_bytes(M, N, K))
+
+
+def linear_plan(M: int, N: int, K: int) -> dict:
+    out = (ctypes.c_int64 * 5)()
+    _lib.check(_lib.load().fp6_linear_plan(M, N, K, out), "fp6_linear_plan")
+    return {"ncol": out[0], "stages": out[1], "grid": out[2], "tiles": out[3], "iters": out[4]}
+
+
+class Workspace:
+    """A zero-initialised device buffer reused across fp6_linear calls on one
+    device and stream (the kernels leave its counters zero after each call)."""
+
+    def __init__(self, device=None):
+        self.device = device
+        self.buf = None
+
+    def get(self, nbytes: int):
+        torch = _torch()
+        if nbytes == 0:
+            return None
+        if self.buf is None or self.buf.numel() < nbytes:
+            self.buf = torch.zeros((max(nbytes, 1 << 20),), dtype=torch.uint8, device=self.device)
+        return self.buf
+
+
+_ws_lock = threading.Lock()
+_default_ws = {}
+
+
+def _default_workspace(device):
+    key = (device.type, device.index, _torch().cuda.current_stream(device).cuda_stream)
+    with _ws_lock:
+        if key not in _default_ws:
+            _default_ws[key] = Workspace(device)
+        return _default_ws[key]
+
+
+def linear(x, packed, scales, N: int, K: int, out=None, workspace: Workspace | None = None):
+    """y[M,N] = x[M,K] . (scales (.) decode(W))^T in fp16 (fp32 accumulation)."""
+    torch = _torch()
+    _need_cuda("x", x, torch.float16, 2)
+    _need_cuda("packed", packed, torch.uint8, 1)
+    _need_cuda("scales", scales, torch.float16, 1)
+    M, K2 = x.shape
+    if K2 != K or scales.shape[0] != N:
+        raise ValueError("shape mismatch between x, scales and (N, K)")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, device=x.device)
+    else:
+        _need_cuda("out", out, torch.float16, 2)
+    need = workspace_bytes(M, N, K)
+    ws = (workspace or _default_workspace(x.device)).get(need)
+    _lib.check(_lib.load().fp6_linear(
+        x.data_ptr(), packed.data_ptr(), scales.data_ptr(), M, N, K, out.data_ptr(),
+        ws.data_ptr() if ws is not None else None, ws.numel() if ws is not None else 0, _stream(x)),
+        "fp6_linear")
+    return out
+
+
+def device_status(device=None) -> int:
+    """Reads and clears the kernels' device error word (0 = OK, 9 = a bounded wait timed out)."""
+    torch = _torch()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    return int(_lib.load().fp6_get_device_status(ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)))
+
+
+class FP6Linear:
+    """A linear layer whose weight is stored as pre-packed FP6 plus fp16 row scales."""
+
+    def __init__(self, packed, scales, N: int, K: int):
+        self.packed, self.scales, self.N, self.K = packed, scales, N, K
+        self.workspace = Workspace(packed.device)
+
+    @classmethod
+    def from_float(cls, W):
+        codes, scales = quantize(W)
+        return cls(prepack(codes), scales, W.shape[0], W.shape[1])
+
+    def __call__(self, x, out=None):
+        return linear(x, self.packed, self.scales, self.N, self.K, out=out, workspace=self.workspace)

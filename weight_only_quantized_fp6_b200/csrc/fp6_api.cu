@@ -1,0 +1,314 @@
+// fp6_api.cu -- the C ABI of libfp6.so (declared in include/fp6.h).
+// Validates arguments on the host, picks the launch configuration, encodes
+// the activation tensor map and launches the kernels on the caller's stream.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "fp6.h"
+#include "fp6_aux_kernels.cuh"
+#include "fp6_linear.cuh"
+
+namespace {
+
+using fp6::LinearShape;
+
+constexpr int kMaxDevices = 64;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+fp6_status check_shape(int64_t N, int64_t K) {
+  if (N < 0 || K < 0) return FP6_ERR_INVALID_ARG;
+  if (N % fp6::kTileRows != 0 || K % fp6::kTileCols != 0) return FP6_ERR_UNSUPPORTED_SHAPE;
+  if (N > (int64_t(1) << 30) || K > (int64_t(1) << 30)) return FP6_ERR_UNSUPPORTED_SHAPE;
+  return FP6_OK;
+}
+
+fp6_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FP6_OK : FP6_ERR_CUDA; }
+
+// ---- per-device cached properties ------------------------------------------
+struct DeviceInfo {
+  int sms = 0;
+  bool attrs_set[5] = {false, false, false, false, false};
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+
+int current_device_sms(int* dev_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  *dev_out = dev;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_dev[dev].sms == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    g_dev[dev].sms = v;
+  }
+  return g_dev[dev].sms;
+}
+
+// ---- tensor-map encoder from the driver (no link-time libcuda dependency) ---
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// ---- launch plan --------------------------------------------------------------
+struct Plan {
+  int ncol = 16;
+  int stages = 0;
+  int grid = 0;
+  int n_tiles = 0, m_tiles = 0, k_tiles = 0;
+  long long tiles = 0;
+  long long total = 0;
+  size_t counter_bytes = 0;
+  size_t partial_bytes = 0;
+};
+
+int pick_ncol(int64_t M) {
+  if (M <= 16) return 16;
+  if (M <= 32) return 32;
+  if (M <= 64) return 64;
+  if (M <= 128) return 128;
+  return 256;
+}
+
+int stages_for(int ncol) {
+  switch (ncol) {
+    case 16: return LinearShape<16>::kStages;
+    case 32: return LinearShape<32>::kStages;
+    case 64: return LinearShape<64>::kStages;
+    case 128: return LinearShape<128>::kStages;
+    default: return LinearShape<256>::kStages;
+  }
+}
+
+bool make_plan(int64_t M, int64_t N, int64_t K, int sms, Plan* pl) {
+  pl->ncol = pick_ncol(M);
+  pl->stages = stages_for(pl->ncol);
+  pl->n_tiles = static_cast<int>(N / fp6::kTileRows);
+  pl->m_tiles = static_cast<int>((M + pl->ncol - 1) / pl->ncol);
+  pl->k_tiles = static_cast<int>(K / fp6::kTileCols);
+  pl->tiles = static_cast<long long>(pl->n_tiles) * pl->m_tiles;
+  pl->total = pl->tiles * pl->k_tiles;
+  if (pl->total <= 0) {
+    pl->grid = 0;
+    return true;
+  }
+  pl->grid = static_cast<int>(std::min<long long>(std::min(sms, fp6::kMaxGrid), pl->total));
+  pl->counter_bytes = fp6::kCounterBytes;
+  pl->partial_bytes = static_cast<size_t>(2) * pl->grid * pl->ncol * 128 * sizeof(float);
+  return true;
+}
+
+template <int NCOL>
+fp6_status launch_linear(const CUtensorMap& map, const fp6::LinearParams& prm, cudaStream_t stream, int dev) {
+  using S = LinearShape<NCOL>;
+  auto kern = fp6::fp6_linear_kernel<NCOL>;
+  const int idx = NCOL == 16 ? 0 : NCOL == 32 ? 1 : NCOL == 64 ? 2 : NCOL == 128 ? 3 : 4;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_dev[dev].attrs_set[idx]) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmemBytes) != cudaSuccess)
+        return FP6_ERR_CUDA;
+      g_dev[dev].attrs_set[idx] = true;
+    }
+  }
+  kern<<<prm.grid, fp6::kLinearThreads, S::kSmemBytes, stream>>>(map, prm);
+  return cuda_status(cudaGetLastError());
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fp6_status_string(fp6_status s) {
+  switch (s) {
+    case FP6_OK: return "FP6_OK";
+    case FP6_ERR_INVALID_ARG: return "FP6_ERR_INVALID_ARG";
+    case FP6_ERR_UNSUPPORTED_SHAPE: return "FP6_ERR_UNSUPPORTED_SHAPE";
+    case FP6_ERR_MISALIGNED: return "FP6_ERR_MISALIGNED";
+    case FP6_ERR_NONFINITE: return "FP6_ERR_NONFINITE";
+    case FP6_ERR_SCALE_RANGE: return "FP6_ERR_SCALE_RANGE";
+    case FP6_ERR_WORKSPACE: return "FP6_ERR_WORKSPACE";
+    case FP6_ERR_CUDA: return "FP6_ERR_CUDA";
+    case FP6_ERR_TIMEOUT: return "FP6_ERR_TIMEOUT";
+  }
+  return "FP6_ERR_UNKNOWN";
+}
+
+size_t fp6_packed_bytes(int64_t N, int64_t K) {
+  if (check_shape(N, K) != FP6_OK) return 0;
+  return static_cast<size_t>(N) * static_cast<size_t>(K) / 4 * 3;
+}
+
+fp6_status fp6_quantize(const float* W, int64_t N, int64_t K, uint8_t* codes, uint16_t* scales,
+                        cudaStream_t stream) {
+  if (N < 0 || K < 0) return FP6_ERR_INVALID_ARG;
+  if (N == 0) return FP6_OK;
+  if (N > INT32_MAX) return FP6_ERR_UNSUPPORTED_SHAPE;
+  if (!scales || (K > 0 && (!W || !codes))) return FP6_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(codes) || !aligned16(scales)) return FP6_ERR_MISALIGNED;
+  const unsigned int zero = 0;
+  cudaError_t e = cudaMemcpyToSymbolAsync(fp6::g_quant_error, &zero, sizeof(zero), 0,
+                                          cudaMemcpyHostToDevice, stream);
+  if (e != cudaSuccess) return FP6_ERR_CUDA;
+  fp6::quantize_kernel<256><<<static_cast<unsigned int>(N), 256, 0, stream>>>(W, K, codes, scales);
+  if (cudaGetLastError() != cudaSuccess) return FP6_ERR_CUDA;
+  unsigned int flags = 0;
+  e = cudaMemcpyFromSymbolAsync(&flags, fp6::g_quant_error, sizeof(flags), 0, cudaMemcpyDeviceToHost, stream);
+  if (e != cudaSuccess) return FP6_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return FP6_ERR_CUDA;
+  if (flags & fp6::kQuantNonfinite) return FP6_ERR_NONFINITE;
+  if (flags & fp6::kQuantScaleRange) return FP6_ERR_SCALE_RANGE;
+  return FP6_OK;
+}
+
+fp6_status fp6_prepack(const uint8_t* codes, int64_t N, int64_t K, void* packed, size_t packed_bytes,
+                       cudaStream_t stream) {
+  fp6_status st = check_shape(N, K);
+  if (st != FP6_OK) return st;
+  if (N == 0 || K == 0) return FP6_OK;
+  if (!codes || !packed) return FP6_ERR_INVALID_ARG;
+  if (packed_bytes < fp6_packed_bytes(N, K)) return FP6_ERR_INVALID_ARG;
+  if (!aligned16(codes) || !aligned16(packed)) return FP6_ERR_MISALIGNED;
+  const int64_t work = N * (K / fp6::kTileCols);
+  const int64_t blocks = (work + 255) / 256;
+  fp6::prepack_kernel<<<static_cast<unsigned int>(blocks), 256, 0, stream>>>(
+      codes, N, K, static_cast<uint8_t*>(packed));
+  return cuda_status(cudaGetLastError());
+}
+
+fp6_status fp6_dequant(const void* packed, const uint16_t* scales, int64_t N, int64_t K, uint16_t* W16,
+                       cudaStream_t stream) {
+  fp6_status st = check_shape(N, K);
+  if (st != FP6_OK) return st;
+  if (N == 0 || K == 0) return FP6_OK;
+  if (!packed || !W16) return FP6_ERR_INVALID_ARG;
+  if (!aligned16(packed) || !aligned16(W16) || (scales && !aligned16(scales))) return FP6_ERR_MISALIGNED;
+  const int64_t work = N * (K / fp6::kTileCols);
+  const int64_t blocks = (work + 255) / 256;
+  fp6::dequant_kernel<<<static_cast<unsigned int>(blocks), 256, 0, stream>>>(
+      static_cast<const uint8_t*>(packed), scales, N, K, W16);
+  return cuda_status(cudaGetLastError());
+}
+
+fp6_status fp6_linear_plan(int64_t M, int64_t N, int64_t K, int64_t out[5]) {
+  if (!out) return FP6_ERR_INVALID_ARG;
+  fp6_status st = check_shape(N, K);
+  if (st != FP6_OK) return st;
+  if (M < 0) return FP6_ERR_INVALID_ARG;
+  if (M > INT32_MAX) return FP6_ERR_UNSUPPORTED_SHAPE;
+  int dev = 0;
+  const int sms = current_device_sms(&dev);
+  if (sms <= 0) return FP6_ERR_CUDA;
+  Plan pl;
+  make_plan(M, N, K, sms, &pl);
+  out[0] = pl.ncol;
+  out[1] = pl.stages;
+  out[2] = pl.grid;
+  out[3] = pl.tiles;
+  out[4] = pl.total;
+  return FP6_OK;
+}
+
+size_t fp6_linear_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (check_shape(N, K) != FP6_OK || M < 0 || M > INT32_MAX) return 0;
+  int dev = 0;
+  const int sms = current_device_sms(&dev);
+  if (sms <= 0) return 0;
+  Plan pl;
+  make_plan(M, N, K, sms, &pl);
+  if (pl.grid == 0) return 0;
+  return pl.counter_bytes + pl.partial_bytes;
+}
+
+fp6_status fp6_linear(const uint16_t* x, const void* packed, const uint16_t* scales, int64_t M, int64_t N,
+                      int64_t K, uint16_t* y, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  fp6_status st = check_shape(N, K);
+  if (st != FP6_OK) return st;
+  if (M < 0) return FP6_ERR_INVALID_ARG;
+  if (M > INT32_MAX) return FP6_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0 || N == 0) return FP6_OK;
+  if (!y) return FP6_ERR_INVALID_ARG;
+  if (!aligned16(y)) return FP6_ERR_MISALIGNED;
+  if (K == 0) {  // empty sum
+    return cuda_status(cudaMemsetAsync(y, 0, static_cast<size_t>(M) * N * sizeof(uint16_t), stream));
+  }
+  if (!x || !packed || !scales) return FP6_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(packed) || !aligned16(scales)) return FP6_ERR_MISALIGNED;
+  int dev = 0;
+  const int sms = current_device_sms(&dev);
+  if (sms <= 0) return FP6_ERR_CUDA;
+  Plan pl;
+  make_plan(M, N, K, sms, &pl);
+  const size_t need = pl.counter_bytes + pl.partial_bytes;
+  if (workspace_bytes < need || (need > 0 && workspace == nullptr)) return FP6_ERR_WORKSPACE;
+  if (need > 0 && !aligned16(workspace)) return FP6_ERR_MISALIGNED;
+
+  EncodeTiledFn encode = get_encode_fn();
+  if (!encode) return FP6_ERR_CUDA;
+  CUtensorMap map;
+  std::memset(&map, 0, sizeof(map));
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * sizeof(uint16_t)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(fp6::kTileCols), static_cast<cuuint32_t>(pl.ncol)};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult cr = encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t*>(x), dims, strides, box, estr,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (cr != CUDA_SUCCESS) return FP6_ERR_CUDA;
+
+  fp6::LinearParams prm;
+  prm.packed = static_cast<const uint8_t*>(packed);
+  prm.scales = scales;
+  prm.y = y;
+  prm.counters = static_cast<uint32_t*>(workspace);
+  prm.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + pl.counter_bytes);
+  prm.M = static_cast<int>(M);
+  prm.N = static_cast<int>(N);
+  prm.K = static_cast<int>(K);
+  prm.n_tiles = pl.n_tiles;
+  prm.m_tiles = pl.m_tiles;
+  prm.k_tiles = pl.k_tiles;
+  prm.total_iters = pl.total;
+  prm.grid = pl.grid;
+  switch (pl.ncol) {
+    case 16: return launch_linear<16>(map, prm, stream, dev);
+    case 32: return launch_linear<32>(map, prm, stream, dev);
+    case 64: return launch_linear<64>(map, prm, stream, dev);
+    case 128: return launch_linear<128>(map, prm, stream, dev);
+    default: return launch_linear<256>(map, prm, stream, dev);
+  }
+}
+
+fp6_status fp6_get_device_status(cudaStream_t stream) {
+  unsigned int word = 0;
+  const unsigned int zero = 0;
+  if (cudaMemcpyFromSymbolAsync(&word, fp6::g_error_word, sizeof(word), 0, cudaMemcpyDeviceToHost, stream) !=
+      cudaSuccess)
+    return FP6_ERR_CUDA;
+  if (cudaMemcpyToSymbolAsync(fp6::g_error_word, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, stream) !=
+      cudaSuccess)
+    return FP6_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return FP6_ERR_CUDA;
+  return (word & fp6::kErrTimeout) ? FP6_ERR_TIMEOUT : FP6_OK;
+}
+
+}  // extern "C"

@@ -16,6 +16,9 @@ activation seed = weight seed + 100 + M.
 """
 from __future__ import annotations
 
+import os
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 
 _GOLDEN = np.uint64(0x9E3779B97F4A7C15)
@@ -85,6 +88,22 @@ def weights(seed: int, N: int, K: int, rows=None, sigma: float = 0.02,
             w[sel] *= np.float32(outlier_mult)
         W[i:j] = w.reshape(j - i, K)
         i = j
+    return W
+
+
+def weights_parallel(seed: int, N: int, K: int, outlier_p: float = 0.0, threads: int = 0) -> np.ndarray:
+    """The full fp32 weight matrix, generated in row blocks on several threads
+    (identical to weights(seed, N, K, outlier_p=...))."""
+    W = np.empty((N, K), dtype=np.float32)
+    threads = threads or min(16, os.cpu_count() or 4)
+    block = max(1, N // (threads * 4))
+
+    def job(r0):
+        r1 = min(N, r0 + block)
+        weights(seed, N, K, rows=range(r0, r1), outlier_p=outlier_p, out=W[r0:r1])
+
+    with ThreadPoolExecutor(threads) as ex:
+        list(ex.map(job, range(0, N, block)))
     return W
 
 
