@@ -134,7 +134,7 @@ fp6_status fp6_linear(const uint16_t *x, const void *packed, const uint16_t *sca
 fp6_status fp6_get_device_status(struct CUstream_st *stream);
 
 /* Launch configuration fp6_linear would use (for tests and benchmarks):
- * out[0] = MMA N-tile (tokens per tile), out[1] = pipeline stages,
+ * out[0] = MMA N-tile (tokens per tile), out[1] = weight pipeline stages,
  * out[2] = persistent CTAs, out[3] = number of (token, row) tiles,
  * out[4] = k-iterations in total.  Returns FP6_OK or an argument error. */
 fp6_status fp6_linear_plan(int64_t M, int64_t N, int64_t K, int64_t out[5]);

@@ -91,11 +91,11 @@ int pick_ncol(int64_t M) {
 
 int stages_for(int ncol) {
   switch (ncol) {
-    case 16: return LinearShape<16>::kStages;
-    case 32: return LinearShape<32>::kStages;
-    case 64: return LinearShape<64>::kStages;
-    case 128: return LinearShape<128>::kStages;
-    default: return LinearShape<256>::kStages;
+    case 16: return LinearShape<16>::kSW;
+    case 32: return LinearShape<32>::kSW;
+    case 64: return LinearShape<64>::kSW;
+    case 128: return LinearShape<128>::kSW;
+    default: return LinearShape<256>::kSW;
   }
 }
 
@@ -120,6 +120,7 @@ bool make_plan(int64_t M, int64_t N, int64_t K, int sms, Plan* pl) {
 template <int NCOL>
 fp6_status launch_linear(const CUtensorMap& map, const fp6::LinearParams& prm, cudaStream_t stream, int dev) {
   using S = LinearShape<NCOL>;
+  static_assert(fp6::kLinearThreads == 704, "launch shape");
   auto kern = fp6::fp6_linear_kernel<NCOL>;
   const int idx = NCOL == 16 ? 0 : NCOL == 32 ? 1 : NCOL == 64 ? 2 : NCOL == 128 ? 3 : 4;
   {
