@@ -124,6 +124,13 @@ size_t fp6_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
  *              only when that size is 0
  * Concurrent calls must not share a workspace.  Deterministic: the same
  * inputs give the same bits on every run.
+ * Launch: programmatic dependent launch.  The kernel may start before the
+ * previous kernel in the stream has finished and begins streaming `packed`
+ * then; x, scales and every output are touched only after that kernel has
+ * completed.  A previous kernel that does not signal early completion (all
+ * other entry points of this library and ordinary kernels) delays the start
+ * until it has finished, so it may write `packed`; a kernel that does signal
+ * early completion must not be the one that writes `packed` just before.
  */
 fp6_status fp6_linear(const uint16_t *x, const void *packed, const uint16_t *scales,
                       int64_t M, int64_t N, int64_t K, uint16_t *y,
@@ -136,7 +143,8 @@ fp6_status fp6_get_device_status(struct CUstream_st *stream);
 /* Launch configuration fp6_linear would use (for tests and benchmarks):
  * out[0] = MMA N-tile (tokens per tile), out[1] = weight pipeline stages,
  * out[2] = persistent CTAs, out[3] = number of (token, row) tiles,
- * out[4] = k-iterations in total.  Returns FP6_OK or an argument error. */
+ * out[4] = pipeline steps in total (a step is one to four 64-column tiles).
+ * Returns FP6_OK or an argument error. */
 fp6_status fp6_linear_plan(int64_t M, int64_t N, int64_t K, int64_t out[5]);
 
 #ifdef __cplusplus

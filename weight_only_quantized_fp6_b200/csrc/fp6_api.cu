@@ -75,8 +75,10 @@ struct Plan {
   int stages = 0;
   int grid = 0;
   int n_tiles = 0, m_tiles = 0, k_tiles = 0;
+  int T = 1;        // 64-column tiles per pipeline step
+  int k_steps = 0;  // steps per (row tile, token tile)
   long long tiles = 0;
-  long long total = 0;
+  long long total = 0;  // steps in all
   size_t counter_bytes = 0;
   size_t partial_bytes = 0;
 };
@@ -87,6 +89,16 @@ int pick_ncol(int64_t M) {
   if (M <= 64) return 64;
   if (M <= 128) return 128;
   return 256;
+}
+
+int tmax_for(int ncol) {
+  switch (ncol) {
+    case 16: return LinearShape<16>::kTMax;
+    case 32: return LinearShape<32>::kTMax;
+    case 64: return LinearShape<64>::kTMax;
+    case 128: return LinearShape<128>::kTMax;
+    default: return LinearShape<256>::kTMax;
+  }
 }
 
 int stages_for(int ncol) {
@@ -106,32 +118,51 @@ bool make_plan(int64_t M, int64_t N, int64_t K, int sms, Plan* pl) {
   pl->m_tiles = static_cast<int>((M + pl->ncol - 1) / pl->ncol);
   pl->k_tiles = static_cast<int>(K / fp6::kTileCols);
   pl->tiles = static_cast<long long>(pl->n_tiles) * pl->m_tiles;
-  pl->total = pl->tiles * pl->k_tiles;
+  // widest step (power of two up to the variant's limit) that divides K/64
+  pl->T = tmax_for(pl->ncol);
+  while (pl->T > 1 && pl->k_tiles % pl->T != 0) pl->T >>= 1;
+  pl->k_steps = pl->k_tiles / pl->T;
+  pl->total = pl->tiles * pl->k_steps;
   if (pl->total <= 0) {
     pl->grid = 0;
     return true;
   }
   pl->grid = static_cast<int>(std::min<long long>(std::min(sms, fp6::kMaxGrid), pl->total));
+  // the decode variants (NCOL <= 64) handle one token tile: NCOL >= M
+  if (pl->ncol <= 64 && pl->m_tiles != 1) return false;
   pl->counter_bytes = fp6::kCounterBytes;
   pl->partial_bytes = static_cast<size_t>(2) * pl->grid * pl->ncol * 128 * sizeof(float);
   return true;
 }
 
+// Launches one variant with programmatic dependent launch: the kernel may
+// begin while the previous kernel in the stream finishes (see the kernel's
+// grid-dependency rules).
 template <int NCOL>
 fp6_status launch_linear(const CUtensorMap& map, const fp6::LinearParams& prm, cudaStream_t stream, int dev) {
-  using S = LinearShape<NCOL>;
-  static_assert(fp6::kLinearThreads == 704, "launch shape");
   auto kern = fp6::fp6_linear_kernel<NCOL>;
+  const int smem = LinearShape<NCOL>::kSmemBytes;
+  const int threads = fp6::kLinearThreads;
   const int idx = NCOL == 16 ? 0 : NCOL == 32 ? 1 : NCOL == 64 ? 2 : NCOL == 128 ? 3 : 4;
   {
     std::lock_guard<std::mutex> lk(g_mu);
     if (!g_dev[dev].attrs_set[idx]) {
-      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmemBytes) != cudaSuccess)
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return FP6_ERR_CUDA;
       g_dev[dev].attrs_set[idx] = true;
     }
   }
-  kern<<<prm.grid, fp6::kLinearThreads, S::kSmemBytes, stream>>>(map, prm);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned int>(prm.grid));
+  cfg.blockDim = dim3(static_cast<unsigned int>(threads));
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, map, prm) != cudaSuccess) return FP6_ERR_CUDA;
   return cuda_status(cudaGetLastError());
 }
 
@@ -277,6 +308,7 @@ fp6_status fp6_linear(const uint16_t* x, const void* packed, const uint16_t* sca
   if (cr != CUDA_SUCCESS) return FP6_ERR_CUDA;
 
   fp6::LinearParams prm;
+  prm.x = x;
   prm.packed = static_cast<const uint8_t*>(packed);
   prm.scales = scales;
   prm.y = y;
@@ -288,7 +320,9 @@ fp6_status fp6_linear(const uint16_t* x, const void* packed, const uint16_t* sca
   prm.n_tiles = pl.n_tiles;
   prm.m_tiles = pl.m_tiles;
   prm.k_tiles = pl.k_tiles;
-  prm.total_iters = pl.total;
+  prm.T = pl.T;
+  prm.k_steps = pl.k_steps;
+  prm.total_steps = pl.total;
   prm.grid = pl.grid;
   switch (pl.ncol) {
     case 16: return launch_linear<16>(map, prm, stream, dev);

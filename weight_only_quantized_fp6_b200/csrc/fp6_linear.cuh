@@ -6,41 +6,56 @@
 // dequantization and the tensor-core product in one kernel, rebuilds FP16
 // weights with bit-parallel SIMT work in registers, and overlaps the two with
 // a software pipeline.  On sm_100a this becomes a warp-specialised persistent
-// kernel.  Per 64-column step ("iteration") of a 128-row weight tile:
+// kernel.  The unit of the pipeline is a "step": T consecutive 64-column tiles
+// of one 128-row weight tile (T = 1, 2 or 4).  Every mbarrier wait or
+// tcgen05.commit costs a warp about 90 cycles and one MMA issue about 50, so
+// per-step synchronisation is amortised over T tiles.
 //
-//   warp 20       weight producer: one 6144-byte bulk copy of the packed tile
-//                 into a smem ring (SW stages);
-//   warp 21       activation producer: one TMA tile copy of x (NCOL rows x 64,
-//                 128-byte swizzle, rows beyond M zero-filled) into a smem ring
-//                 of R stages;
-//   warps 8..19   three dequant warpgroups taking every third iteration: each
-//                 thread owns one weight row (its TMEM lane), reads its 48
-//                 packed bytes, splices 64 fp16 weights (decode * 2^-12) and
-//                 stores them into a ring of R TMEM slots (tcgen05.st);
-//   warps 0..3    MMA issuers.  tcgen05.mma (M = 128, K = 16) costs a warp
-//                 about 47 cycles to issue whatever N is, so at small N one
-//                 issuer cannot keep up with HBM; NISS issuers each take a
-//                 k-slice of every step (K/NISS) into their own fp32
-//                 accumulator in TMEM, A from the TMEM slot, B = x from smem;
-//   warps 4..7    the epilogue warpgroup: per segment (the iterations of one
-//                 tile this CTA owns), tcgen05.ld of the NISS accumulators,
+//   warp 20       weight producer: one bulk copy of the step's T packed tiles
+//                 (contiguous, T * 6144 bytes) into a smem ring (SW stages);
+//   warp 21       activation producer into a ring of RX stages: for one token
+//                 tile (M <= NCOL <= 64) 16-byte cp.async copies of the M valid
+//                 rows (x stays off the TMA engine, which the weight stream keeps
+//                 busy); otherwise T TMA tile copies (NCOL rows x 64, 128-byte
+//                 swizzle, rows beyond M zero-filled);
+//   warps 8..19   three dequant warpgroups taking every third step: each thread
+//                 owns one weight row (its TMEM lane), reads its 48 packed bytes
+//                 per tile, splices 64 fp16 weights (decode * 2^-12) and stores
+//                 them into the step's TMEM slot (tcgen05.st);
+//   warps 0..3    MMA issuers: NISS warps each take a k-slice of every tile
+//                 (tcgen05.mma M = 128, N = NCOL, K = 16; A from the TMEM slot,
+//                 B = x from smem) into their own fp32 accumulator in TMEM;
+//   warps 4..7    the epilogue warpgroup: per segment (the steps of one tile
+//                 that this CTA owns), tcgen05.ld of the NISS accumulators,
 //                 summed in a fixed order, * scale * 2^12, fp16 store, or the
 //                 split-K partial and fix-up.
 //
-// An iteration's x stage and TMEM slot are released together by the issuers'
-// commits on one "consumed" barrier.  Every mbarrier has consumers that wait on
-// its phases in order (a ring slot always belongs to the same dequant group:
-// SW and R are multiples of the group count), so no wait can alias a phase two
+// Three rings: packed weights (SW smem stages, filled by the weight
+// producer, released by the dequant group), x (RX smem stages, released by
+// the issuers' commits) and dequantized weights (R TMEM slots, released by the
+// issuers' commits).  Every mbarrier's consumers wait on its phases in order
+// (a weight stage or TMEM slot always belongs to the same dequant group: SW
+// and R are multiples of the group count), so no wait can alias a phase two
 // steps ahead.
 //
-// Work split: the (token tile, row tile, 64-column step) iterations are laid
-// out row-tile major and cut into G contiguous, equal ranges, one per
-// persistent CTA (G = number of SMs).  A row tile whose steps span several
-// CTAs is finished by the last of them to arrive (atomic counter), which sums
-// the partials in CTA order: results are deterministic and no CTA waits on
+// Work split: the (token tile, row tile, step) iterations are laid out
+// row-tile major and cut into G contiguous, equal ranges, one per persistent
+// CTA (G = number of SMs).  A row tile whose steps span several CTAs is
+// finished by the last of them to arrive (atomic counter), which sums the
+// partials in CTA order: results are deterministic and no CTA waits on
 // another.  A split tile's counter is indexed by its first contributing CTA,
 // which is unique among split tiles and below G, so the counters occupy a
 // fixed region of the workspace that no partial ever overlaps.
+//
+// Launch: programmatic dependent launch.  The kernel may start while the
+// previous kernel in the stream is finishing: barrier set-up, TMEM allocation
+// and the stream of packed weights overlap its tail.  Reads of x and scales
+// and every write (y, partials, counters) come after griddepcontrol.wait, i.e.
+// after the previous kernel has completed and its writes are visible.  A
+// previous kernel that never signals early completion (every kernel of this
+// library but this one, and ordinary kernels) only lets this kernel start once
+// it has finished, so packed weights written by it are seen too; packed
+// weights must not be produced by a kernel that does signal early completion.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -64,46 +79,57 @@ constexpr uint32_t kTmemCols = 512;
 template <int NCOL>
 struct LinearShape {
   static_assert(NCOL == 16 || NCOL == 32 || NCOL == 64 || NCOL == 128 || NCOL == 256, "NCOL");
-  static constexpr int kXBytes = NCOL * 128;   // NCOL rows x 64 fp16, 128-byte swizzled
+  static constexpr int kTMax = (NCOL <= 32) ? 4 : (NCOL <= 128) ? 2 : 1;   // tiles per step, at most
+  static constexpr int kXTile = NCOL * 128;                 // NCOL rows x 64 fp16, 128-byte swizzled
+  static constexpr int kXStage = kTMax * kXTile;
+  static constexpr int kWStage = kTMax * kTileBytes;
   static constexpr int kIssuers = (NCOL <= 32) ? 4 : (NCOL == 64) ? 2 : 1;
-  static constexpr int kR = (NCOL <= 64) ? 12 : (NCOL == 128) ? 6 : 3;      // x stages = TMEM slots
-  static constexpr int kSW = (NCOL == 16) ? 27 : (NCOL == 32) ? 24 : 18;   // weight stages
-  static constexpr int kDCol = kR * 32;        // accumulators after the TMEM slot ring
-  static constexpr int kWOff = kR * kXBytes;   // weight ring after the x ring
-  static constexpr int kBarOff = kWOff + kSW * kTileBytes;
+  static constexpr int kRX = (NCOL == 16) ? 8 : (NCOL <= 64) ? 4 : 3;     // x stages (>= 3)
+  static constexpr int kSW = (NCOL <= 32) ? 6 : (NCOL == 64) ? 12 : (NCOL == 128) ? 9 : 18;  // weight stages
+  static constexpr int kR = (kTMax == 4) ? 3 : 6;           // TMEM slots
+  static constexpr int kSlotCols = kTMax * 32;              // TMEM columns of one slot
+  static constexpr int kDCol = kR * kSlotCols;              // accumulators after the slots
+  static constexpr int kWOff = kRX * kXStage;               // weight ring after the x ring
+  static constexpr int kBarOff = kWOff + kSW * kWStage;
+  static constexpr int kNumBars = 2 * kSW + 2 * kRX + 2 * kR + 5;
   static constexpr int kBarrierBytes = 1024;
   static constexpr int kSmemBytes = kBarOff + kBarrierBytes + 1024;  // + alignment slack
-  static_assert(kXBytes % 1024 == 0 && kTileBytes % 1024 == 0, "1024-byte aligned stages");
+  static_assert(kXTile % 1024 == 0 && kTileBytes % 1024 == 0, "1024-byte aligned tiles");
   static_assert(kSW % kDeqGroups == 0 && kR % kDeqGroups == 0, "ring slots owned by one group");
   static_assert(kDCol + kIssuers * NCOL <= static_cast<int>(kTmemCols), "TMEM budget");
-  static_assert((2 * kSW + 3 * kR + 6) * 8 + 32 <= kBarrierBytes, "barrier area");
+  static_assert(kNumBars * 8 + 32 <= kBarrierBytes, "barrier area");
+  static_assert(kNumBars <= kLinearThreads, "one thread per barrier at set-up");
   static_assert(kSmemBytes <= 232448, "shared memory");
 };
 
 struct LinearParams {
+  const uint16_t* x;     // [M,K] fp16 (read directly by the decode kernel; the prefill kernel uses TMA)
   const uint8_t* packed;
   const uint16_t* scales;
   uint16_t* y;
   float* partials;       // [2*G][NCOL][128] fp32
   uint32_t* counters;    // [kMaxGrid], indexed by a split tile's first CTA; zero on entry and exit
   int M, N, K;
-  int n_tiles, m_tiles, k_tiles;
-  long long total_iters;
+  int n_tiles, m_tiles, k_tiles;   // k_tiles = K / 64
+  int T;                           // tiles per step (divides k_tiles, <= kTMax)
+  int k_steps;                     // k_tiles / T
+  long long total_steps;           // n_tiles * m_tiles * k_steps
   int grid;
 };
 
-// First iteration of CTA c's range.
+// First step of CTA c's range.
 __host__ __device__ __forceinline__ long long range_begin(int c, long long total, int G) {
   return static_cast<long long>(c) * total / G;
 }
-// CTA whose range holds iteration i:  max{c : range_begin(c) <= i}.
+// CTA whose range holds step i:  max{c : range_begin(c) <= i}.
 __host__ __device__ __forceinline__ int range_owner(long long i, long long total, int G) {
   return static_cast<int>(((i + 1) * G + total - 1) / total - 1);
 }
-// Partial slot of CTA c's segment in tile t: 0 for the tile its range starts
-// in, 1 for the tile its range ends in (only those two can be partial).
-__host__ __device__ __forceinline__ int partial_slot(int c, long long t, long long total, int G, int KT) {
-  return 2 * c + ((range_begin(c, total, G) / KT == t) ? 0 : 1);
+// Partial slot of CTA c's segment in tile t (KS steps per tile): 0 for the
+// tile its range starts in, 1 for the tile its range ends in (only those two
+// can be partial).
+__host__ __device__ __forceinline__ int partial_slot(int c, long long t, long long total, int G, int KS) {
+  return 2 * c + ((range_begin(c, total, G) / KS == t) ? 0 : 1);
 }
 
 // Every lane of the warp waits; the warp continues only if all lanes saw the
@@ -113,20 +139,20 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
   return __all_sync(0xffffffffu, ok) != 0;
 }
 
-// Walks the CTA's iterations: the 64-column step k and the tile's (row tile,
-// token tile) coordinates, advanced without divisions.
-struct IterCursor {
-  int k, nt, mt;
-  int KT, MT;
-  __device__ __forceinline__ IterCursor(long long it0, int KT_, int MT_) : KT(KT_), MT(MT_) {
-    const long long tile = it0 / KT_;
-    k = static_cast<int>(it0 - tile * KT_);
+// Walks the CTA's steps: the step index within the tile and the tile's (row
+// tile, token tile) coordinates, advanced without divisions.
+struct StepCursor {
+  int ks, nt, mt;
+  int KS, MT;
+  __device__ __forceinline__ StepCursor(long long s0, int KS_, int MT_) : KS(KS_), MT(MT_) {
+    const long long tile = s0 / KS_;
+    ks = static_cast<int>(s0 - tile * KS_);
     nt = static_cast<int>(tile / MT_);
     mt = static_cast<int>(tile - static_cast<long long>(nt) * MT_);
   }
   __device__ __forceinline__ void next() {
-    if (++k == KT) {
-      k = 0;
+    if (++ks == KS) {
+      ks = 0;
       if (++mt == MT) {
         mt = 0;
         ++nt;
@@ -135,25 +161,38 @@ struct IterCursor {
   }
 };
 
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void fence_acq_rel_gpu() {
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
+}
+
 template <int NCOL>
 __global__ void __launch_bounds__(kLinearThreads, 1)
     fp6_linear_kernel(const __grid_constant__ CUtensorMap tmap_x, const LinearParams p) {
   using S = LinearShape<NCOL>;
   constexpr int kR = S::kR;
+  constexpr int kRX = S::kRX;
   constexpr int kSW = S::kSW;
   constexpr int kISS = S::kIssuers;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* wfull = reinterpret_cast<uint64_t*>(smem + S::kBarOff);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBarOff);
+  uint64_t* wfull = bars;
   uint64_t* wempty = wfull + kSW;
   uint64_t* xfull = wempty + kSW;
-  uint64_t* afull = xfull + kR;
-  uint64_t* consumed = afull + kR;                // x stage + TMEM slot free (issuer commits)
+  uint64_t* xempty = xfull + kRX;                 // x stage free (issuer commits)
+  uint64_t* afull = xempty + kRX;
+  uint64_t* consumed = afull + kR;                // TMEM slot free (issuer commits)
   uint64_t* dfull = consumed + kR;
   uint64_t* dempty = dfull + 1;
   uint64_t* done = dempty + 1;
   uint64_t* epi = done + 1;                       // [2]: fix-up meeting of the first / last split segment
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(epi + 2);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + S::kNumBars);
   volatile int* s_last = reinterpret_cast<volatile int*>(tmem_holder + 1);  // [2]
   volatile int* s_abort = s_last + 2;
   volatile int* s_never = s_abort + 1;            // an abort flag nothing raises (final drains)
@@ -162,118 +201,187 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
   const int lane = threadIdx.x & 31;
   const int G = p.grid;
   const int c = blockIdx.x;
-  const long long total = p.total_iters;
+  const long long total = p.total_steps;
+  const int KS = p.k_steps;
+  const int T = p.T;
   const int KT = p.k_tiles;
   const int MT = p.m_tiles;
-  const long long it0 = range_begin(c, total, G);
-  const long long it1 = range_begin(c + 1, total, G);
-  const int n_local = static_cast<int>(it1 - it0);
-  const long long tile_first = it0 / KT;
-  const long long tile_last = (it1 - 1) / KT;
+  const long long s0 = range_begin(c, total, G);
+  const long long s1 = range_begin(c + 1, total, G);
+  const int n_local = static_cast<int>(s1 - s0);
+  const long long tile_first = s0 / KS;
+  const long long tile_last = (s1 - 1) / KS;
 
+  // Let the next kernel in the stream be scheduled as early as possible.
+  grid_launch_dependents();
+
+  // Barrier set-up, one thread per barrier.
+  if (threadIdx.x < S::kNumBars) {
+    const int b = threadIdx.x;
+    const int bx = 2 * kSW, ba = bx + 2 * kRX, bd = ba + 2 * kR;
+    uint32_t count = 1;                                       // wfull, xfull: producer arrive + tx
+    if (b >= kSW && b < bx) count = 4;                        // wempty: the reading group's 4 warps
+    else if (b >= bx + kRX && b < ba) count = kISS;           // xempty: issuer commits
+    else if (b >= ba && b < ba + kR) count = 4;               // afull: the writing group
+    else if (b >= ba + kR && b < bd) count = kISS;            // consumed: issuer commits
+    else if (b == bd) count = kISS;                           // dfull
+    else if (b == bd + 1) count = 4;                          // dempty: epilogue warps
+    else if (b == bd + 2) count = kISS;                       // done
+    else if (b >= bd + 3) count = 4;                          // epi[0], epi[1]
+    mbar_init(smem_u32(&bars[b]), count);
+    fence_barrier_init();
+  }
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kSW; ++s) {
-      mbar_init(smem_u32(&wfull[s]), 1);
-      mbar_init(smem_u32(&wempty[s]), 4);      // the 4 warps of the group that read it
-    }
-    for (int s = 0; s < kR; ++s) {
-      mbar_init(smem_u32(&xfull[s]), 1);
-      mbar_init(smem_u32(&afull[s]), 4);       // the 4 warps of the group that wrote it
-      mbar_init(smem_u32(&consumed[s]), kISS); // one commit per issuer
-    }
-    mbar_init(smem_u32(dfull), kISS);
-    mbar_init(smem_u32(dempty), 4);
-    mbar_init(smem_u32(done), kISS);
-    mbar_init(smem_u32(&epi[0]), 4);
-    mbar_init(smem_u32(&epi[1]), 4);
     s_last[0] = 0;
     s_last[1] = 0;
     *s_abort = 0;
     *s_never = 0;
-    fence_barrier_init();
-    fence_proxy_async_smem();
   }
   if (warp == kXProdWarp && lane == 0) prefetch_tensormap(&tmap_x);
   if (warp == 0) {
     tmem_alloc(smem_u32(tmem_holder), kTmemCols);
     tmem_relinquish();
   }
+  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
+  // Producer and issuer loops run on whole warps: every lane waits on the
+  // barriers (the warp stays converged) and lane 0 alone issues the copy, MMA
+  // or commit.
   if (warp == kWProdWarp) {
     // ---------------- weight producer ----------------
-    if (lane == 0) {
-      const uint64_t pol = policy_evict_first();
-      IterCursor cur(it0, KT, MT);
-      int issued = 0;
-      for (int li = 0; li < n_local; ++li, cur.next()) {
-        const int s = li % kSW;
-        if (li >= kSW && !wait_bounded(smem_u32(&wempty[s]), ((li / kSW) - 1) & 1, s_abort)) break;
+    const uint64_t pol = policy_evict_first();
+    StepCursor cur(s0, KS, MT);
+    const uint32_t bytes = static_cast<uint32_t>(T) * kTileBytes;
+    int issued = 0;
+    for (int li = 0; li < n_local; ++li, cur.next()) {
+      const int s = li % kSW;
+      if (li >= kSW && !warp_wait(smem_u32(&wempty[s]), ((li / kSW) - 1) & 1, s_abort)) break;
+      if (lane == 0) {
         const uint32_t fb = smem_u32(&wfull[s]);
-        mbar_arrive_expect_tx(fb, kTileBytes);
-        bulk_load(smem_u32(smem + S::kWOff + s * kTileBytes),
-                  p.packed + (static_cast<long long>(cur.nt) * KT + cur.k) * kTileBytes, kTileBytes, fb, pol);
-        ++issued;
+        mbar_arrive_expect_tx(fb, bytes);
+        bulk_load(smem_u32(smem + S::kWOff + s * S::kWStage),
+                  p.packed + (static_cast<long long>(cur.nt) * KT + static_cast<long long>(cur.ks) * T) * kTileBytes,
+                  bytes, fb, pol);
       }
-      // Leave no copy in flight: the last copy issued into every stage has landed.
-      for (int li = issued > kSW ? issued - kSW : 0; li < issued; ++li)
-        wait_bounded(smem_u32(&wfull[li % kSW]), (li / kSW) & 1, s_never);
+      __syncwarp();
+      ++issued;
     }
+    // Leave no copy in flight: the last copy issued into every stage has landed.
+    for (int li = issued > kSW ? issued - kSW : 0; li < issued; ++li)
+      warp_wait(smem_u32(&wfull[li % kSW]), (li / kSW) & 1, s_never);
   } else if (warp == kXProdWarp) {
     // ---------------- activation producer ----------------
-    if (lane == 0) {
+    grid_dependency_wait();                  // x is written by earlier work in the stream
+    if constexpr (NCOL <= 64) {
+      // One token tile (M <= NCOL): LSU copies keep x off the TMA engine,
+      // which the weight stream keeps busy.  Rows at or beyond M are never
+      // loaded, so every stage is zeroed once; each step copies the M valid
+      // rows of its T x tiles in 16-byte chunks straight into the
+      // 128-byte-swizzled layout (chunk ch of row r at (ch ^ (r % 8)) * 16).
+      for (int i = lane; i < kRX * S::kXStage / 16; i += 32)
+        *reinterpret_cast<uint4*>(smem + i * 16) = make_uint4(0u, 0u, 0u, 0u);
+      __syncwarp();
+      constexpr int kDepth = (kRX - 2 < 3) ? kRX - 2 : 3;   // steps in flight besides the newest
+      const int chunks_per_row = T * 8;
+      const int chunks = p.M * chunks_per_row;
+      int ks = static_cast<int>(s0 - tile_first * KS);
+      int signalled = 0;
+      int issued = 0;
+      for (int li = 0; li < n_local; ++li, ks = (ks + 1 == KS) ? 0 : ks + 1) {
+        const int s = li % kRX;
+        if (li >= kRX && !warp_wait(smem_u32(&xempty[s]), ((li / kRX) - 1) & 1, s_abort)) break;
+        uint8_t* stage = smem + s * S::kXStage;
+        const uint16_t* src0 = p.x + static_cast<long long>(ks) * T * kTileCols;
+        for (int idx = lane; idx < chunks; idx += 32) {
+          const int r = idx / chunks_per_row;
+          const int rem = idx - r * chunks_per_row;
+          const int t = rem >> 3, ch = rem & 7;
+          cp_async_16(smem_u32(stage + t * S::kXTile + r * 128 + ((ch ^ (r & 7)) << 4)),
+                      src0 + static_cast<long long>(r) * p.K + t * kTileCols + ch * 8);
+        }
+        cp_async_commit();
+        ++issued;
+        if (issued - signalled > kDepth) {
+          // the oldest step's copies have landed: make them visible to the tensor core
+          cp_async_wait<kDepth>();
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&xfull[signalled % kRX]));
+          ++signalled;
+        }
+      }
+      cp_async_wait<0>();
+      fence_proxy_async_smem();
+      __syncwarp();
+      for (; signalled < issued; ++signalled)
+        if (lane == 0) mbar_arrive(smem_u32(&xfull[signalled % kRX]));
+    } else {
       const uint64_t pol = policy_evict_last();
-      IterCursor cur(it0, KT, MT);
+      StepCursor cur(s0, KS, MT);
+      const uint32_t bytes = static_cast<uint32_t>(T) * S::kXTile;
       int issued = 0;
       for (int li = 0; li < n_local; ++li, cur.next()) {
-        const int s = li % kR;
-        if (li >= kR && !wait_bounded(smem_u32(&consumed[s]), ((li / kR) - 1) & 1, s_abort)) break;
-        const uint32_t fb = smem_u32(&xfull[s]);
-        mbar_arrive_expect_tx(fb, S::kXBytes);
-        tma_load_2d(smem_u32(smem + s * S::kXBytes), &tmap_x, fb, cur.k * kTileCols, cur.mt * NCOL, pol);
+        const int s = li % kRX;
+        if (li >= kRX && !warp_wait(smem_u32(&xempty[s]), ((li / kRX) - 1) & 1, s_abort)) break;
+        if (lane == 0) {
+          const uint32_t fb = smem_u32(&xfull[s]);
+          mbar_arrive_expect_tx(fb, bytes);
+          for (int t = 0; t < T; ++t)
+            tma_load_2d(smem_u32(smem + s * S::kXStage + t * S::kXTile), &tmap_x, fb,
+                        (cur.ks * T + t) * kTileCols, cur.mt * NCOL, pol);
+        }
+        __syncwarp();
         ++issued;
       }
-      for (int li = issued > kR ? issued - kR : 0; li < issued; ++li)
-        wait_bounded(smem_u32(&xfull[li % kR]), (li / kR) & 1, s_never);
+      for (int li = issued > kRX ? issued - kRX : 0; li < issued; ++li)
+        warp_wait(smem_u32(&xfull[li % kRX]), (li / kRX) & 1, s_never);
     }
   } else if (warp < kISS) {
-    // ---------------- MMA issuer `warp`: k-slice [warp*4/kISS, (warp+1)*4/kISS) of every step ----------------
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_f16_f32(128, NCOL);
-      constexpr int kSlice = 4 / kISS;
-      const int kk0 = warp * kSlice;
-      const uint32_t d_tmem = tmem + S::kDCol + warp * NCOL;
-      int sg = 0;
-      int k = static_cast<int>(it0 - tile_first * KT);
-      for (int li = 0; li < n_local; ++li, k = (k + 1 == KT) ? 0 : k + 1) {
-        const bool seg_first = (li == 0) || (k == 0);
-        const bool seg_last = (li == n_local - 1) || (k == KT - 1);
-        const int s = li % kR;
-        if (seg_first && sg > 0 && !wait_bounded(smem_u32(dempty), (sg - 1) & 1, s_abort)) break;
-        if (!wait_bounded(smem_u32(&xfull[s]), (li / kR) & 1, s_abort)) break;
-        if (!wait_bounded(smem_u32(&afull[s]), (li / kR) & 1, s_abort)) break;
+    // ---------------- MMA issuer `warp`: k-slice [warp*4/kISS, (warp+1)*4/kISS) of every tile ----------------
+    constexpr uint32_t idesc = idesc_f16_f32(128, NCOL);
+    constexpr int kSlice = 4 / kISS;
+    const int kk0 = warp * kSlice;
+    const uint32_t d_tmem = tmem + S::kDCol + warp * NCOL;
+    int sg = 0;
+    int ks = static_cast<int>(s0 - tile_first * KS);
+    for (int li = 0; li < n_local; ++li, ks = (ks + 1 == KS) ? 0 : ks + 1) {
+      const bool seg_first = (li == 0) || (ks == 0);
+      const bool seg_last = (li == n_local - 1) || (ks == KS - 1);
+      const int s = li % kR;
+      const int sx = li % kRX;
+      if (seg_first && sg > 0 && !warp_wait(smem_u32(dempty), (sg - 1) & 1, s_abort)) break;
+      if (!warp_wait(smem_u32(&xfull[sx]), (li / kRX) & 1, s_abort)) break;
+      if (!warp_wait(smem_u32(&afull[s]), (li / kR) & 1, s_abort)) break;
+      if (lane == 0) {
         tc_fence_after();
-        const uint64_t bdesc = smem_desc_sw128(smem_u32(smem + s * S::kXBytes));
+        const uint64_t bdesc0 = smem_desc_sw128(smem_u32(smem + sx * S::kXStage));
+        const uint32_t a0 = tmem + s * S::kSlotCols;
+        for (int t = 0; t < T; ++t) {
+          // B descriptor of tile t: start address advances by kXTile bytes (>> 4)
+          const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(t * (S::kXTile >> 4));
 #pragma unroll
-        for (int j = 0; j < kSlice; ++j) {
-          const int kk = kk0 + j;
-          // K = 16 per MMA: 8 TMEM columns of A, 32 bytes along the swizzled B rows
-          mma_f16_ts(d_tmem, tmem + s * 32 + kk * 8, bdesc + static_cast<uint64_t>(kk * 2), idesc,
-                     (seg_first && j == 0) ? 0u : 1u);
+          for (int j = 0; j < kSlice; ++j) {
+            const int kk = kk0 + j;
+            // K = 16 per MMA: 8 TMEM columns of A, 32 bytes along the swizzled B rows
+            mma_f16_ts(d_tmem, a0 + t * 32 + kk * 8, bdesc + static_cast<uint64_t>(kk * 2), idesc,
+                       (seg_first && t == 0 && j == 0) ? 0u : 1u);
+          }
         }
+        tc_commit(smem_u32(&xempty[sx]));
         tc_commit(smem_u32(&consumed[s]));
-        if (seg_last) {
-          tc_commit(smem_u32(dfull));
-          ++sg;
-        }
+        if (seg_last) tc_commit(smem_u32(dfull));
       }
-      // All issued MMAs have finished before TMEM is released.
-      tc_commit(smem_u32(done));
-      wait_bounded(smem_u32(done), 0, s_never);
+      __syncwarp();
+      if (seg_last) ++sg;
     }
+    // All issued MMAs have finished before TMEM is released.
+    if (lane == 0) tc_commit(smem_u32(done));
+    __syncwarp();
+    warp_wait(smem_u32(done), 0, s_never);
   } else if (warp >= kFirstDeqWarp) {
     // ---------------- dequant warpgroups ----------------
     const int g = (warp - kFirstDeqWarp) >> 2;
@@ -284,14 +392,17 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
       const int sw = li % kSW;
       const int s = li % kR;
       if (!warp_wait(smem_u32(&wfull[sw]), (li / kSW) & 1, s_abort)) break;
-      uint32_t lo[8], hi[4], w[32];
-      load_row_fragments(smem + S::kWOff + sw * kTileBytes, r, lo, hi);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&wempty[sw]));
       if (li >= kR && !warp_wait(smem_u32(&consumed[s]), ((li / kR) - 1) & 1, s_abort)) break;
       tc_fence_after();
-      splice_row(lo, hi, w);
-      tmem_st_32x32b_x32(tmem + lane_base + s * 32, w);
+      const uint8_t* wst = smem + S::kWOff + sw * S::kWStage;
+      for (int t = 0; t < T; ++t) {
+        uint32_t lo[8], hi[4], w[32];
+        load_row_fragments(wst + t * kTileBytes, r, lo, hi);
+        splice_row(lo, hi, w);
+        tmem_st_32x32b_x32(tmem + lane_base + s * S::kSlotCols + t * 32, w);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&wempty[sw]));   // smem fragments read
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -299,6 +410,7 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
     }
   } else if (warp >= kEpiWarp && warp < kEpiWarp + 4) {
     // ---------------- epilogue warpgroup: segments in order ----------------
+    grid_dependency_wait();                  // y, partials and counters may be in use before this kernel
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const bool leader = (warp == kEpiWarp) && lane == 0;
@@ -313,8 +425,8 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
       const int m0 = mt * NCOL;
       const int mcount = min(NCOL, p.M - m0);
       const float mul = __half2float(__ushort_as_half(p.scales[n])) * 4096.0f;
-      const int c_lo = range_owner(tile * KT, total, G);
-      const int c_hi = range_owner(tile * KT + KT - 1, total, G);
+      const int c_lo = range_owner(tile * KS, total, G);
+      const int c_hi = range_owner(tile * KS + KS - 1, total, G);
       const bool split = c_lo != c_hi;
       const int which = (tile == tile_first) ? 0 : 1;   // this CTA's first or last segment
       float* part = p.partials + static_cast<long long>(2 * c + which) * NCOL * 128;
@@ -336,7 +448,7 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
         }
         if (split) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) part[(c0 + j) * 128 + r] = acc[j];
+          for (int j = 0; j < 8; ++j) __stcg(part + (c0 + j) * 128 + r, acc[j]);
         } else {
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
@@ -346,33 +458,32 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
         }
       }
       if (split) {
-        // Publish this CTA's partial, then count arrivals; the last CTA of the
-        // tile sums every partial in CTA order.  The group's warps meet on an
-        // mbarrier (bounded wait), never on bar.sync, so an aborted warp cannot
-        // strand the others.  Each of the CTA's (at most two) split segments
-        // has its own meeting barrier.
+        // Publish this CTA's partial (release), count arrivals; the last CTA of
+        // the tile (acquire) sums every partial in CTA order.  The group's warps
+        // meet on an mbarrier (bounded wait), never on bar.sync, so an aborted
+        // warp cannot strand the others.  Each of the CTA's (at most two) split
+        // segments has its own meeting barrier.
         const uint32_t eb = smem_u32(&epi[which]);
-        __threadfence();
         __syncwarp();
         if (lane == 0) mbar_arrive(eb);
         if (!warp_wait(eb, 0, s_abort)) break;
         if (leader) {
-          __threadfence();
+          fence_acq_rel_gpu();
           const unsigned int prev = atomicAdd(&p.counters[c_lo], 1u);
+          fence_acq_rel_gpu();
           s_last[which] = (prev == static_cast<unsigned int>(c_hi - c_lo)) ? 1 : 0;
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(eb);
         if (!warp_wait(eb, 1, s_abort)) break;
         if (s_last[which]) {
-          __threadfence();
           for (int c0 = 0; c0 < mcount; c0 += 8) {
             float acc[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
             for (int cc = c_lo; cc <= c_hi; ++cc) {
               const float* src = p.partials +
-                                 static_cast<long long>(partial_slot(cc, tile, total, G, KT)) * NCOL * 128 +
+                                 static_cast<long long>(partial_slot(cc, tile, total, G, KS)) * NCOL * 128 +
                                  c0 * 128 + r;
               float v[8];
 #pragma unroll
