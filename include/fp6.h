@@ -140,6 +140,27 @@ fp6_status fp6_linear(const uint16_t *x, const void *packed, const uint16_t *sca
  * runs out (returns FP6_ERR_TIMEOUT then, else FP6_OK).  Synchronizes `stream`. */
 fp6_status fp6_get_device_status(struct CUstream_st *stream);
 
+/*
+ * fp6_linear_noalloc -- fp6_linear for callers that cannot allocate device
+ * memory while the layer runs (for example a plugin inside an engine that owns
+ * all device memory, or a latency-critical loop where cudaMalloc, which may
+ * synchronize the device, is not allowed).  The FP6-LLM pages have no
+ * counterpart: this is a convenience of this library.
+ *   Same arguments and result as fp6_linear, without the workspace: the
+ *   scratch lives in a fixed 16 MiB array inside the library's device image,
+ *   present on every GPU that loads the library until the process exits.
+ *   Problems whose fp6_linear_workspace_bytes exceed 16 MiB (on a 148-SM B200,
+ *   M > 64) return FP6_ERR_WORKSPACE; use fp6_linear for them.
+ *   The first call on each device looks up the array's device address, so make
+ *   that first call before capturing a stream.  Each call clears the counters
+ *   it needs with cudaMemsetAsync on `stream`; it never allocates or frees.
+ *   All calls on a device share the one array: calls that may overlap on the
+ *   GPU (different streams without ordering between them) race and give wrong
+ *   results.
+ */
+fp6_status fp6_linear_noalloc(const uint16_t *x, const void *packed, const uint16_t *scales,
+                              int64_t M, int64_t N, int64_t K, uint16_t *y, struct CUstream_st *stream);
+
 /* Launch configuration fp6_linear would use (for tests and benchmarks):
  * out[0] = MMA N-tile (tokens per tile), out[1] = weight pipeline stages,
  * out[2] = persistent CTAs, out[3] = number of (token, row) tiles,

@@ -346,4 +346,60 @@ fp6_status fp6_get_device_status(cudaStream_t stream) {
   return (word & fp6::kErrTimeout) ? FP6_ERR_TIMEOUT : FP6_OK;
 }
 
+// ---- allocation-free variant -------------------------------------------------
+// Some callers cannot allocate device memory when they run the layer: a plugin
+// inside an engine that owns every byte of device memory, or a latency-bound
+// loop where cudaMalloc (which may synchronize the device) is not allowed.
+// fp6_linear_noalloc gives them the same layer with its scratch (split-K
+// counters and partial sums) in a fixed array that lives in this library's
+// device image on every GPU that loads it.
+}  // extern "C"
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;   // 16 MiB per device
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+void* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+// Device address of the scratch array on the current device, looked up once
+// per device (the array's host-side name is only a stand-in and must never be
+// handed to a kernel).
+fp6_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FP6_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) return FP6_ERR_CUDA;
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return FP6_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+fp6_status fp6_linear_noalloc(const uint16_t* x, const void* packed, const uint16_t* scales, int64_t M, int64_t N,
+                              int64_t K, uint16_t* y, cudaStream_t stream) {
+  fp6_status st = check_shape(N, K);
+  if (st != FP6_OK) return st;
+  if (M < 0) return FP6_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return FP6_OK;
+  const size_t need = fp6_linear_workspace_bytes(M, N, K);
+  if (need > kNoAllocScratchBytes) return FP6_ERR_WORKSPACE;  // beyond the fixed scratch: use fp6_linear
+  void* scratch = nullptr;
+  st = noalloc_scratch(&scratch);
+  if (st != FP6_OK) return st;
+  if (need > 0) {
+    // The array keeps the previous call's contents: the split-K counters must
+    // start at zero, so clear them on the caller's stream first.
+    if (cudaMemsetAsync(scratch, 0, fp6::kCounterBytes, stream) != cudaSuccess) return FP6_ERR_CUDA;
+  }
+  return fp6_linear(x, packed, scales, M, N, K, y, scratch, kNoAllocScratchBytes, stream);
+}
+
 }  // extern "C"
