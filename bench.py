@@ -19,6 +19,7 @@ import argparse
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -44,6 +45,36 @@ def wbytes(N, K):
 def algo_bytes(M, N, K):
     """Algorithmic bytes of one launch: packed weights + fp16 scales + fp16 activations."""
     return 0.75 * N * K + 2 * N + 2 * M * K
+
+
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "fp6_linear_kernel_llama70b_o_proj_decode.md")
+
+
+def kernel_source_hash() -> str:
+    """First 16 hex digits of the SHA-256 over the library's CUDA sources, sorted by name."""
+    import hashlib
+    csrc = os.path.join(ROOT, "weight_only_quantized_fp6_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes (read + write) of one launch from the committed ncu summary, or
+    None when that capture was taken of a different kernel source."""
+    if not os.path.exists(PROFILE_SUMMARY):
+        return None
+    fields = {}
+    for line in open(PROFILE_SUMMARY):
+        m = re.match(r"^(kernel_source_sha256|dram_bytes_per_launch|captured_launch_M):\s*(\S+)", line)
+        if m:
+            fields[m.group(1)] = m.group(2)
+    if fields.get("kernel_source_sha256") != kernel_source_hash() or "dram_bytes_per_launch" not in fields:
+        return None
+    return {"bytes": int(fields["dram_bytes_per_launch"]), "M": int(fields.get("captured_launch_M", 0))}
 
 
 def read_peaks():
@@ -285,6 +316,7 @@ def run_fp6(args, world, rank, local):
     avg_launch_ms = elapsed_ms / launches
     achieved = float(algo.mean() / (avg_launch_ms / 1e3) / 1e9)
     peaks = read_peaks()
+    prof = profiled_traffic()
 
     # Per-M breakdown (outside the timed region): a graph of 2*copies launches
     # of one M, timed as a whole.
@@ -361,7 +393,11 @@ def run_fp6(args, world, rank, local):
                 "parallelism": f"independent replicas x{world}" if world > 1 else "single GPU",
             },
             "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+                         "frac": round(achieved / peaks["hbm_gbs"], 4),
+                         "traffic": prof["bytes"] if prof else None,
+                         "traffic_note": (f"ncu dram read+write of one M={prof['M']} launch "
+                                          f"(algorithmic {algo_bytes(prof['M'], N_DIM, K_DIM):.0f} B)")
+                         if prof else "no ncu capture of this kernel source",
                          "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs)",
                          "kernel": "fp6_linear_kernel<16>"},
             "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
