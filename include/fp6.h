@@ -76,15 +76,16 @@ fp6_status fp6_quantize(const float *W, int64_t N, int64_t K,
 
 /*
  * fp6_prepack -- bit-level pre-packing (TC-FPx article: weights reorganised
- * before inference, each 6-bit weight split into 2-bit and 4-bit pieces that
- * are stored in aligned 32-bit words, fragments reordered so that the
- * run-time rebuild is parallel).  Layout version 1:
+ * before inference, each 6-bit weight cut into pieces stored in aligned
+ * 32-bit words, fragments reordered so that the run-time rebuild is
+ * parallel).  Layout version 2, cut for the sm_100a instruction that converts
+ * two byte-held e3m2 codes (low six bits of each byte) to two fp16 values:
  *   tiles of 128 rows x 64 columns, tile (nt, kt) at byte (nt*(K/64)+kt)*6144;
- *   inside a tile, row r owns 8 lo words L_q at byte (q/4)*2048 + r*16 + (q%4)*4
- *   and 4 hi words H_p at byte 4096 + r*16 + p*4.  Tile column kk gives pair
- *   j = kk/2, half h = kk%2; code bits 3..0 go to L_{j/4} bits 4(j%4)+16h ..+3;
- *   code bit 4 to H_{j/8} bit 2(j%8)+16h; code bit 5 to H_{j/8} bit
- *   (2(j%8)+3+16h) mod 32.  Words are little-endian.
+ *   inside a tile, row r owns 12 words F_w at byte (w/4)*2048 + r*16 + (w%4)*4.
+ *   Tile column kk is position i = kk%16 of group g = kk/16 (words F_{3g..3g+2}):
+ *   i < 12: the whole code in bits 8b..8b+5 of F_{3g+i/4}, b = i%4;
+ *   i >= 12: b = i-12, code bits 2j and 2j+1 (j = 0,1,2) in bits 8b+6 and
+ *   8b+7 of F_{3g+j}.  Words are little-endian.
  *   codes   [N,K] uint8, device (bits 7..6 ignored)
  *   packed  device buffer of packed_bytes >= fp6_packed_bytes(N,K), written
  */

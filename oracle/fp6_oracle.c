@@ -24,7 +24,8 @@
  *   f16 rounding        pinned: numpy float16 conversion (library routine)
  *   quantize            pinned: exact brute-force argmin, round trip, error
  *                       bound, CUDA's own fp6 conversion routine
- *   prepack / unpack    pinned: bit-splice decode of the packed words gives the
+ *   prepack / unpack    pinned: a numpy reading of the packed words (byte
+ *                       containers plus gathered top bits) gives the
  *                       closed-form fp16 pattern; one-hot probe; round trip
  *   dequant             pinned: closed form of decode*scale rounded by numpy
  *   linear              pinned: exact rational dot products (tiny shapes),
@@ -186,34 +187,60 @@ int oracle_quantize(const float *W, int64_t N, int64_t K, uint8_t *codes, uint16
 }
 
 /* ------------------------------------------------------------------------ */
-/* Prepack / unpack: 2+4 bit split into 32-bit-aligned fragment streams      */
+/* Prepack / unpack: bit split into 32-bit-aligned fragment words            */
 /* ------------------------------------------------------------------------ */
 
-/* Packed layout (version 1).  W is cut into tiles of 128 rows x 64 columns,
- * stored tile after tile with the column-tile index fastest:
+/* Packed layout (version 2).  The pages cut each 6-bit weight into pieces held
+ * in aligned 32-bit words so that registers rebuild many weights per
+ * operation; the cut and the order are left open.  This layout is cut for a
+ * converter that turns two bytes, each holding one code in its low six bits,
+ * into two fp16 values and ignores each byte's top two bits: twelve of every
+ * sixteen codes stay whole in the low six bits of a byte, and the other four
+ * are cut into three 2-bit pieces stored in those bytes' top two bits.
+ *
+ * W is cut into tiles of 128 rows x 64 columns, stored tile after tile with
+ * the column-tile index fastest:
  *     tile (nt, kt) at byte (nt * (K/64) + kt) * 6144.
- * Inside a tile, row r (0..127) owns twelve 32-bit words:
- *     lo words L_q, q = 0..7, at byte (q/4)*2048 + r*16 + (q%4)*4
- *     hi words H_p, p = 0..3, at byte 4096 + r*16 + p*4
- * Column kk (0..63) of the tile belongs to pair j = kk/2, half h = kk%2.
- * The code's low four bits (e1 e0 m1 m0) sit in L_{j/4} at bit 4*(j%4) + 16*h.
- * The code's top two bits sit in H_{j/8}, with i = j%8:
- *     e2 (code bit 4) at bit 2*i + 16*h,
- *     s  (code bit 5) at bit (2*i + 3 + 16*h) mod 32.
- * Byte order is little-endian (bit b of a word is bit b%8 of byte b/8). */
+ * Inside a tile, row r (0..127) owns twelve 32-bit words F_w, w = 0..11,
+ *     F_w at byte (w/4)*2048 + r*16 + (w%4)*4.
+ * Column kk (0..63) of the tile belongs to group g = kk/16 (words F_{3g},
+ * F_{3g+1}, F_{3g+2}), position i = kk%16 in the group:
+ *     i < 12: the whole code in bits 8b..8b+5 of F_{3g + i/4}, b = i%4;
+ *     i >= 12: b = i - 12; code bits 2j and 2j+1 (j = 0, 1, 2) in bits 8b+6
+ *              and 8b+7 of F_{3g + j}.
+ * Byte order is little-endian (bit t of a word is bit t%8 of byte t/8). */
 static inline int64_t tile_base(int64_t n, int64_t k, int64_t K)
 {
     return ((n / 128) * (K / 64) + (k / 64)) * 6144;
 }
 
-static inline void put_bit(uint8_t *buf, int64_t word_byte, int bit, int value)
+static inline int64_t word_byte(int64_t base, int r, int w)
 {
-    if (value) buf[word_byte + bit / 8] |= (uint8_t)(1u << (bit % 8));
+    return base + (w / 4) * 2048 + r * 16 + (w % 4) * 4;
 }
 
-static inline int get_bit(const uint8_t *buf, int64_t word_byte, int bit)
+static inline void put_bit(uint8_t *buf, int64_t wbyte, int bit, int value)
 {
-    return (buf[word_byte + bit / 8] >> (bit % 8)) & 1;
+    if (value) buf[wbyte + bit / 8] |= (uint8_t)(1u << (bit % 8));
+}
+
+static inline int get_bit(const uint8_t *buf, int64_t wbyte, int bit)
+{
+    return (buf[wbyte + bit / 8] >> (bit % 8)) & 1;
+}
+
+/* Where bit t (0..5) of the code at tile row r, tile column kk lives:
+ * the word's byte offset and the bit within that word. */
+static inline void code_bit_place(int64_t base, int r, int kk, int t, int64_t *wbyte, int *bit)
+{
+    int g = kk / 16, i = kk % 16;
+    if (i < 12) {
+        *wbyte = word_byte(base, r, 3 * g + i / 4);
+        *bit = 8 * (i % 4) + t;
+    } else {
+        *wbyte = word_byte(base, r, 3 * g + t / 2);
+        *bit = 8 * (i - 12) + 6 + t % 2;
+    }
 }
 
 int oracle_prepack(const uint8_t *codes, int64_t N, int64_t K, uint8_t *packed)
@@ -225,15 +252,12 @@ int oracle_prepack(const uint8_t *codes, int64_t N, int64_t K, uint8_t *packed)
         for (int64_t k = 0; k < K; ++k) {
             uint8_t c = codes[n * K + k] & 0x3F;
             int64_t base = tile_base(n, k, K);
-            int r = (int)(n % 128), kk = (int)(k % 64);
-            int j = kk / 2, h = kk % 2;
-            int q = j / 4, p = j / 8, i = j % 8;
-            int64_t lo_word = base + (q / 4) * 2048 + r * 16 + (q % 4) * 4;
-            int64_t hi_word = base + 4096 + r * 16 + p * 4;
-            int lo_bit = 4 * (j % 4) + 16 * h;
-            for (int b = 0; b < 4; ++b) put_bit(packed, lo_word, lo_bit + b, (c >> b) & 1);
-            put_bit(packed, hi_word, 2 * i + 16 * h, (c >> 4) & 1);
-            put_bit(packed, hi_word, (2 * i + 3 + 16 * h) % 32, (c >> 5) & 1);
+            for (int t = 0; t < 6; ++t) {
+                int64_t wb;
+                int bit;
+                code_bit_place(base, (int)(n % 128), (int)(k % 64), t, &wb, &bit);
+                put_bit(packed, wb, bit, (c >> t) & 1);
+            }
         }
     }
     return ORC_OK;
@@ -246,16 +270,13 @@ int oracle_unpack(const uint8_t *packed, int64_t N, int64_t K, uint8_t *codes)
     for (int64_t n = 0; n < N; ++n) {
         for (int64_t k = 0; k < K; ++k) {
             int64_t base = tile_base(n, k, K);
-            int r = (int)(n % 128), kk = (int)(k % 64);
-            int j = kk / 2, h = kk % 2;
-            int q = j / 4, p = j / 8, i = j % 8;
-            int64_t lo_word = base + (q / 4) * 2048 + r * 16 + (q % 4) * 4;
-            int64_t hi_word = base + 4096 + r * 16 + p * 4;
-            int lo_bit = 4 * (j % 4) + 16 * h;
             uint8_t c = 0;
-            for (int b = 0; b < 4; ++b) c |= (uint8_t)(get_bit(packed, lo_word, lo_bit + b) << b);
-            c |= (uint8_t)(get_bit(packed, hi_word, 2 * i + 16 * h) << 4);
-            c |= (uint8_t)(get_bit(packed, hi_word, (2 * i + 3 + 16 * h) % 32) << 5);
+            for (int t = 0; t < 6; ++t) {
+                int64_t wb;
+                int bit;
+                code_bit_place(base, (int)(n % 128), (int)(k % 64), t, &wb, &bit);
+                c |= (uint8_t)(get_bit(packed, wb, bit) << t);
+            }
             codes[n * K + k] = c;
         }
     }

@@ -12,9 +12,11 @@
 #include "fp6.h"
 #include "fp6_aux_kernels.cuh"
 #include "fp6_linear.cuh"
+#include "fp6_linear_decode.cuh"
 
 namespace {
 
+using fp6::DecodeShape;
 using fp6::LinearShape;
 
 constexpr int kMaxDevices = 64;
@@ -33,7 +35,7 @@ fp6_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FP6_OK : FP6_E
 // ---- per-device cached properties ------------------------------------------
 struct DeviceInfo {
   int sms = 0;
-  bool attrs_set[5] = {false, false, false, false, false};
+  bool attrs_set[7] = {false, false, false, false, false, false, false};
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -91,10 +93,12 @@ int pick_ncol(int64_t M) {
   return 256;
 }
 
+// Token tiles of up to 32 columns run the decode kernel (fp6_linear_decode.cuh),
+// wider ones the general kernel (fp6_linear.cuh).
 int tmax_for(int ncol) {
   switch (ncol) {
-    case 16: return LinearShape<16>::kTMax;
-    case 32: return LinearShape<32>::kTMax;
+    case 16: return DecodeShape<16>::kTMax;
+    case 32: return DecodeShape<32>::kTMax;
     case 64: return LinearShape<64>::kTMax;
     case 128: return LinearShape<128>::kTMax;
     default: return LinearShape<256>::kTMax;
@@ -103,8 +107,8 @@ int tmax_for(int ncol) {
 
 int stages_for(int ncol) {
   switch (ncol) {
-    case 16: return LinearShape<16>::kSW;
-    case 32: return LinearShape<32>::kSW;
+    case 16: return DecodeShape<16>::kSW;
+    case 32: return DecodeShape<32>::kSW;
     case 64: return LinearShape<64>::kSW;
     case 128: return LinearShape<128>::kSW;
     default: return LinearShape<256>::kSW;
@@ -155,6 +159,34 @@ fp6_status launch_linear(const CUtensorMap& map, const fp6::LinearParams& prm, c
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned int>(prm.grid));
   cfg.blockDim = dim3(static_cast<unsigned int>(threads));
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, map, prm) != cudaSuccess) return FP6_ERR_CUDA;
+  return cuda_status(cudaGetLastError());
+}
+
+// The decode kernel (one token tile of at most 32 columns), launched the same way.
+template <int NCOL>
+fp6_status launch_decode(const CUtensorMap& map, const fp6::LinearParams& prm, cudaStream_t stream, int dev) {
+  auto kern = fp6::fp6_linear_decode_kernel<NCOL>;
+  const int smem = DecodeShape<NCOL>::kSmemBytes;
+  const int idx = NCOL == 16 ? 5 : 6;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_dev[dev].attrs_set[idx]) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return FP6_ERR_CUDA;
+      g_dev[dev].attrs_set[idx] = true;
+    }
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned int>(prm.grid));
+  cfg.blockDim = dim3(static_cast<unsigned int>(fp6::kDecThreads));
   cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -294,19 +326,6 @@ fp6_status fp6_linear(const uint16_t* x, const void* packed, const uint16_t* sca
   if (workspace_bytes < need || (need > 0 && workspace == nullptr)) return FP6_ERR_WORKSPACE;
   if (need > 0 && !aligned16(workspace)) return FP6_ERR_MISALIGNED;
 
-  EncodeTiledFn encode = get_encode_fn();
-  if (!encode) return FP6_ERR_CUDA;
-  CUtensorMap map;
-  std::memset(&map, 0, sizeof(map));
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * sizeof(uint16_t)};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(fp6::kTileCols), static_cast<cuuint32_t>(pl.ncol)};
-  const cuuint32_t estr[2] = {1, 1};
-  CUresult cr = encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t*>(x), dims, strides, box, estr,
-                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (cr != CUDA_SUCCESS) return FP6_ERR_CUDA;
-
   fp6::LinearParams prm;
   prm.x = x;
   prm.packed = static_cast<const uint8_t*>(packed);
@@ -324,9 +343,22 @@ fp6_status fp6_linear(const uint16_t* x, const void* packed, const uint16_t* sca
   prm.k_steps = pl.k_steps;
   prm.total_steps = pl.total;
   prm.grid = pl.grid;
+  EncodeTiledFn encode = get_encode_fn();
+  if (!encode) return FP6_ERR_CUDA;
+  CUtensorMap map;
+  std::memset(&map, 0, sizeof(map));
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * sizeof(uint16_t)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(fp6::kTileCols), static_cast<cuuint32_t>(pl.ncol)};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult cr = encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t*>(x), dims, strides, box, estr,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (cr != CUDA_SUCCESS) return FP6_ERR_CUDA;
+
   switch (pl.ncol) {
-    case 16: return launch_linear<16>(map, prm, stream, dev);
-    case 32: return launch_linear<32>(map, prm, stream, dev);
+    case 16: return launch_decode<16>(map, prm, stream, dev);
+    case 32: return launch_decode<32>(map, prm, stream, dev);
     case 64: return launch_linear<64>(map, prm, stream, dev);
     case 128: return launch_linear<128>(map, prm, stream, dev);
     default: return launch_linear<256>(map, prm, stream, dev);

@@ -89,13 +89,13 @@ __global__ void __launch_bounds__(256) prepack_kernel(const uint8_t* __restrict_
 #pragma unroll
     for (int b = 0; b < 16; ++b) c[16 * v + b] = static_cast<uint8_t>(w[b >> 2] >> (8 * (b & 3)));
   }
-  uint32_t lo[8], hi[4];
-  pack_row(c, lo, hi);
+  uint32_t F[kRowWords];
+  pack_row(c, F);
   uint8_t* tile = packed + ((n / kTileRows) * KT + kt) * kTileBytes;
   const int r = static_cast<int>(n % kTileRows);
-  *reinterpret_cast<uint4*>(tile + r * 16) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-  *reinterpret_cast<uint4*>(tile + 2048 + r * 16) = make_uint4(lo[4], lo[5], lo[6], lo[7]);
-  *reinterpret_cast<uint4*>(tile + kLoBytes + r * 16) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+#pragma unroll
+  for (int u = 0; u < 3; ++u)
+    *reinterpret_cast<uint4*>(tile + u * 2048 + r * 16) = make_uint4(F[4 * u], F[4 * u + 1], F[4 * u + 2], F[4 * u + 3]);
 }
 
 // One thread per (row, tile): splice the row's 64 weights and write them as
@@ -110,10 +110,10 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* __restrict_
   const int64_t kt = idx / N;
   const int64_t n = idx % N;
   const uint8_t* tile = packed + ((n / kTileRows) * KT + kt) * kTileBytes;
-  uint32_t lo[8], hi[4], w[32];
-  load_row_fragments(tile, static_cast<int>(n % kTileRows), lo, hi);
-  splice_row(lo, hi, w);
-  const float mul = 4096.0f * (scales ? __half2float(__ushort_as_half(scales[n])) : 1.0f);
+  uint32_t F[kRowWords], w[32];
+  load_row_words(tile, static_cast<int>(n % kTileRows), F);
+  splice_row(F, w);
+  const float mul = scales ? __half2float(__ushort_as_half(scales[n])) : 1.0f;
   uint16_t* dst = W16 + n * K + kt * kTileCols;
 #pragma unroll
   for (int v = 0; v < 8; ++v) {

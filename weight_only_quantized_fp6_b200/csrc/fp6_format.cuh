@@ -1,31 +1,30 @@
 // fp6_format.cuh -- FP6 (e3m2) encoding on the device: the packed layout,
-// the bit-splice rebuild of fp16 weights, and the quantizer's rounding.
+// the register rebuild of fp16 weights, and the quantizer's rounding.
 //
 // e3m2 code (low 6 bits of a byte): s = bit 5, e = bits 4..2 (bias 3),
 // m = bits 1..0.  Value (-1)^s 2^(e-3)(1+m/4), or (-1)^s 2^-2 (m/4) for e = 0.
+// Every value is exact in fp16.
 //
-// Rebuild identity.  Put s at fp16 bit 15 and the five bits e,m at fp16 bits
-// 12..8: the fp16 exponent field then equals e and the top two mantissa bits
-// equal m, so the half is exactly decode(c) * 2^-12 -- e = 0 codes land on
-// fp16 subnormals with the right value.  The layer multiplies by 2^12 once,
-// folded into the per-row scale in the fp32 epilogue.
+// Rebuild.  The TC-FPx article ("kernel solution redesign") cuts each 6-bit
+// weight into pieces held in aligned 32-bit words and rebuilds FP16 weights
+// in registers, many per operation.  sm_100a converts a pair of e3m2 codes to
+// an fp16 pair in one instruction (cvt.rn.f16x2.e3m2x2), reading the low six
+// bits of each of the two bytes and ignoring their top two bits; the layout
+// below is cut for it.  Of every 16 codes of a row, 12 stay whole in the low
+// six bits of a byte and are converted straight from the loaded words; the
+// other 4 are cut into three 2-bit pieces kept in the top two bits of those
+// bytes and gathered with two masked merges and three shifts into one more
+// word of byte containers.  Per row of a tile: 32 conversions and 20 integer
+// operations for 64 weights.
 //
-// Split (TC-FPx article, "kernel solution redesign": each 6-bit weight is cut
-// into a 2-bit and a 4-bit piece held in aligned 32-bit words, rebuilt in
-// parallel in registers).  Here the 4-bit piece is e1 e0 m1 m0, which already
-// sits at fp16 bits 11..8 after a shift; the 2-bit piece is (s, e2), targets
-// fp16 bits 15 and 12.  Two halves are produced per 32-bit operation.
-//
-// Packed layout (version 1), per tile of 128 rows x 64 columns (6144 bytes,
-// tiles stored row-tile major, column-tile minor): row r owns lo words L_q
-// (q = 0..7) at byte (q/4)*2048 + r*16 + (q%4)*4 and hi words H_p (p = 0..3)
-// at byte 4096 + r*16 + p*4, so a warp reading 16 bytes per row touches 512
-// consecutive bytes (no bank conflicts).  Pair j (columns 2j, 2j+1) of the row
-// is rebuilt as
-//     rotl(H_{j/8}, 12 - 2(j%8)) & 0x90009000   |   shift(L_{j/4}, 8 - 4(j%4)) & 0x0F000F00
-// i.e. the nibble of column 2j+h sits at L bits 4(j%4)+16h, e2 at H bit
-// 2(j%8)+16h and s at H bit (2(j%8)+3+16h) mod 32.  The eight rotations
-// place the 16 two-bit fields of a hi word onto disjoint bit sets.
+// Packed layout (version 2), per tile of 128 rows x 64 columns (6144 bytes,
+// tiles stored row-tile major, column-tile minor): row r owns words F_w
+// (w = 0..11) at byte (w/4)*2048 + r*16 + (w%4)*4, so a warp reading 16 bytes
+// per row touches 512 consecutive bytes (no bank conflicts).  Column kk of
+// the tile is position i = kk%16 of group g = kk/16 (words F_{3g..3g+2}):
+//     i < 12: the whole code in bits 8b..8b+5 of F_{3g + i/4}, b = i%4;
+//     i >= 12: b = i - 12; code bits 2j, 2j+1 (j = 0..2) in bits 8b+6, 8b+7
+//              of F_{3g + j}.
 #pragma once
 #include <cstdint>
 #include <cuda_fp16.h>
@@ -35,48 +34,62 @@ namespace fp6 {
 constexpr int kTileRows = 128;
 constexpr int kTileCols = 64;
 constexpr int kTileBytes = 6144;
-constexpr int kLoBytes = 4096;
+constexpr int kRowWords = 12;
 
-// Rebuild the 64 fp16 weights (as 32 fp16x2 words, low half = even column) of
-// one row of one tile from its 8 lo words and 4 hi words.
-__device__ __forceinline__ void splice_row(const uint32_t (&lo)[8], const uint32_t (&hi)[4],
-                                           uint32_t (&out)[32]) {
+// Two e3m2 codes (the low six bits of bytes 0 and 1, resp. 2 and 3, of w) to
+// two fp16 pairs: o0 = (byte 0, byte 1), o1 = (byte 2, byte 3), low half first.
+__device__ __forceinline__ void cvt_e3m2x4(uint32_t w, uint32_t& o0, uint32_t& o1) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "cvt.rn.f16x2.e3m2x2 %0, l;\n\tcvt.rn.f16x2.e3m2x2 %1, h;\n\t}"
+      : "=r"(o0), "=r"(o1)
+      : "r"(w));
+}
+
+// Rebuild the 64 fp16 weights (as 32 fp16x2 words, low half = even column)
+// of one row of one tile from its 12 words: decode(c) exactly.
+__device__ __forceinline__ void splice_row(const uint32_t (&F)[kRowWords], uint32_t (&out)[32]) {
 #pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    const uint32_t h = hi[j >> 3];
-    const uint32_t hr = __funnelshift_l(h, h, (12 - 2 * (j & 7)) & 31);
-    const uint32_t l = lo[j >> 2];
-    const int t = j & 3;
-    const uint32_t lr = (t < 2) ? (l << (8 - 4 * t)) : (l >> (4 * t - 8));
-    out[j] = (hr & 0x90009000u) | (lr & 0x0F000F00u);
+  for (int g = 0; g < 4; ++g) {
+    const uint32_t f0 = F[3 * g], f1 = F[3 * g + 1], f2 = F[3 * g + 2];
+    // cut codes: top bits of f2 (code bits 5,4), f1 (3,2), f0 (1,0) -> bits 5..0
+    const uint32_t u1 = (f2 & 0xC0C0C0C0u) | ((f1 >> 2) & 0x3F3F3F3Fu);
+    const uint32_t u2 = (u1 & 0xF0F0F0F0u) | ((f0 >> 4) & 0x0F0F0F0Fu);
+    const uint32_t t = u2 >> 2;
+    cvt_e3m2x4(f0, out[8 * g + 0], out[8 * g + 1]);
+    cvt_e3m2x4(f1, out[8 * g + 2], out[8 * g + 3]);
+    cvt_e3m2x4(f2, out[8 * g + 4], out[8 * g + 5]);
+    cvt_e3m2x4(t, out[8 * g + 6], out[8 * g + 7]);
   }
 }
 
-// Load the row's fragments from a tile that starts at `tile` (shared or
+// Load the row's 12 words from a tile that starts at `tile` (shared or
 // global memory, 16-byte aligned).
-__device__ __forceinline__ void load_row_fragments(const uint8_t* tile, int r, uint32_t (&lo)[8],
-                                                   uint32_t (&hi)[4]) {
-  const uint4 a = *reinterpret_cast<const uint4*>(tile + r * 16);
-  const uint4 b = *reinterpret_cast<const uint4*>(tile + 2048 + r * 16);
-  const uint4 c = *reinterpret_cast<const uint4*>(tile + kLoBytes + r * 16);
-  lo[0] = a.x; lo[1] = a.y; lo[2] = a.z; lo[3] = a.w;
-  lo[4] = b.x; lo[5] = b.y; lo[6] = b.z; lo[7] = b.w;
-  hi[0] = c.x; hi[1] = c.y; hi[2] = c.z; hi[3] = c.w;
+__device__ __forceinline__ void load_row_words(const uint8_t* tile, int r, uint32_t (&F)[kRowWords]) {
+#pragma unroll
+  for (int u = 0; u < 3; ++u) {
+    const uint4 a = *reinterpret_cast<const uint4*>(tile + u * 2048 + r * 16);
+    F[4 * u + 0] = a.x;
+    F[4 * u + 1] = a.y;
+    F[4 * u + 2] = a.z;
+    F[4 * u + 3] = a.w;
+  }
 }
 
-// Pack 64 codes (columns 0..63 of one tile row) into the row's words.
-__device__ __forceinline__ void pack_row(const uint8_t (&c)[64], uint32_t (&lo)[8], uint32_t (&hi)[4]) {
+// Pack 64 codes (columns 0..63 of one tile row) into the row's 12 words.
+__device__ __forceinline__ void pack_row(const uint8_t (&c)[64], uint32_t (&F)[kRowWords]) {
 #pragma unroll
-  for (int q = 0; q < 8; ++q) lo[q] = 0;
-#pragma unroll
-  for (int p = 0; p < 4; ++p) hi[p] = 0;
+  for (int w = 0; w < kRowWords; ++w) F[w] = 0;
 #pragma unroll
   for (int kk = 0; kk < 64; ++kk) {
-    const int j = kk >> 1, h = kk & 1, i = j & 7;
+    const int g = kk >> 4, i = kk & 15;
     const uint32_t code = c[kk] & 0x3Fu;
-    lo[j >> 2] |= (code & 0xFu) << (4 * (j & 3) + 16 * h);
-    hi[j >> 3] |= ((code >> 4) & 1u) << (2 * i + 16 * h);
-    hi[j >> 3] |= ((code >> 5) & 1u) << ((2 * i + 3 + 16 * h) & 31);
+    if (i < 12) {
+      F[3 * g + (i >> 2)] |= code << (8 * (i & 3));
+    } else {
+      const int b = i - 12;
+#pragma unroll
+      for (int j = 0; j < 3; ++j) F[3 * g + j] |= ((code >> (2 * j)) & 3u) << (8 * b + 6);
+    }
   }
 }
 

@@ -20,14 +20,14 @@
 //                 swizzle, rows beyond M zero-filled);
 //   warps 8..19   three dequant warpgroups taking every third step: each thread
 //                 owns one weight row (its TMEM lane), reads its 48 packed bytes
-//                 per tile, splices 64 fp16 weights (decode * 2^-12) and stores
+//                 per tile, rebuilds 64 fp16 weights (decode(c), exact) and stores
 //                 them into the step's TMEM slot (tcgen05.st);
 //   warps 0..3    MMA issuers: NISS warps each take a k-slice of every tile
 //                 (tcgen05.mma M = 128, N = NCOL, K = 16; A from the TMEM slot,
 //                 B = x from smem) into their own fp32 accumulator in TMEM;
 //   warps 4..7    the epilogue warpgroup: per segment (the steps of one tile
 //                 that this CTA owns), tcgen05.ld of the NISS accumulators,
-//                 summed in a fixed order, * scale * 2^12, fp16 store, or the
+//                 summed in a fixed order, * scale, fp16 store, or the
 //                 split-K partial and fix-up.
 //
 // Three rings: packed weights (SW smem stages, filled by the weight
@@ -396,9 +396,9 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
       tc_fence_after();
       const uint8_t* wst = smem + S::kWOff + sw * S::kWStage;
       for (int t = 0; t < T; ++t) {
-        uint32_t lo[8], hi[4], w[32];
-        load_row_fragments(wst + t * kTileBytes, r, lo, hi);
-        splice_row(lo, hi, w);
+        uint32_t F[kRowWords], w[32];
+        load_row_words(wst + t * kTileBytes, r, F);
+        splice_row(F, w);
         tmem_st_32x32b_x32(tmem + lane_base + s * S::kSlotCols + t * 32, w);
       }
       __syncwarp();
@@ -424,7 +424,7 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
       const int n = nt * kTileRows + r;
       const int m0 = mt * NCOL;
       const int mcount = min(NCOL, p.M - m0);
-      const float mul = __half2float(__ushort_as_half(p.scales[n])) * 4096.0f;
+      const float mul = __half2float(__ushort_as_half(p.scales[n]));
       const int c_lo = range_owner(tile * KS, total, G);
       const int c_hi = range_owner(tile * KS + KS - 1, total, G);
       const bool split = c_lo != c_hi;
