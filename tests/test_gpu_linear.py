@@ -221,3 +221,29 @@ def test_workspace_reused_across_shapes(fp6, orc):
         y = fp6.linear(as_f16(x), packed, scales, N, K, workspace=ws)
         codes_o, scales_o = orc.quantize(W)
         parity.assert_close(bits16(y), orc.linear(x, codes_o, scales_o, nthreads=8), f"N={N} K={K} M={M}")
+
+
+@pytest.fixture(scope="module")
+def split_heavy_layer(orc):
+    N, K = 21504, 7168
+    W = parity.gen_weights_parallel(4242, N, K, 0.0)
+    codes_o, scales_o = orc.quantize(W)
+    return W, codes_o, scales_o
+
+
+@pytest.mark.parametrize("M", [1, 16, 32])
+def test_split_heavy_layer_every_row(fp6, orc, split_heavy_layer, M):
+    """OPT-30B QKV shape (N = 21504, K = 7168): every persistent CTA covers
+    more than one row tile, so ranges hold up to three segments and every
+    split tile is finished by another CTA than the ones that published its
+    partials.  The whole output is compared, not a sample, so a row tile whose
+    fix-up went wrong cannot hide."""
+    from weight_only_quantized_fp6_b200 import inputs
+    N, K = 21504, 7168
+    W, codes_o, scales_o = split_heavy_layer
+    codes, scales, packed = gpu_layer(fp6, W)
+    x = inputs.activations(4243 + M, M, K)
+    y = bits16(fp6.linear(as_f16(x), packed, scales, N, K))
+    assert np.array_equal(codes.cpu().numpy(), codes_o)
+    ref = orc.linear(x, codes_o, scales_o, nthreads=16)
+    parity.assert_close(y, ref, f"N={N} K={K} M={M}")

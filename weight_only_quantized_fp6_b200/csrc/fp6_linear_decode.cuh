@@ -110,7 +110,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   uint64_t* slotfree = xempty + kRX;              // [6]: a group's MMAs on the slot are done
   uint64_t* dfull = slotfree + S::kSlots;         // [2]: a segment's accumulators are complete
   uint64_t* dempty = dfull + 2;                   // [2]: the epilogue has read them
-  uint64_t* epi = dempty + 2;                     // [2]: fix-up meetings
+  uint64_t* epi = dempty + 2;                     // [2]: fix-up meeting (epi[0] only)
   uint64_t* done = epi + 2;                       // every MMA finished (before TMEM release)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + S::kNumBars);
   volatile int* s_last = reinterpret_cast<volatile int*>(tmem_holder + 1);  // [2]
@@ -284,10 +284,17 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     }
   } else if (warp >= kDecEpiWarp && warp < kDecEpiWarp + 4) {
     // ---------------- epilogue warpgroup: segments in order ----------------
+    // A split row tile is finished by its first CTA c_lo, which reaches the
+    // tile at the end of its range; every later contributor reaches it at the
+    // start of its own range, publishes its partial there (release add on the
+    // tile's counter) and moves on.  The finishing CTA waits for those
+    // partials and sums them (in CTA order) while its own MMAs still run, so
+    // the end of its range costs one TMEM read and the store of y.  Each
+    // epilogue warp of a contributor releases its 32 rows with one add, so the
+    // counter reaches 4 per contributor.
     grid_dependency_wait();                  // y, partials and counters may be in use before this kernel
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
-    const bool leader = (warp == kDecEpiWarp) && lane == 0;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const int mcount = min(NCOL, p.M);
     for (int sg = 0; sg < nseg; ++sg) {
@@ -295,16 +302,37 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       const int set = sg & 1;
       int a, b;
       segment_range(sg, tile_first, s0, KS, n_local, &a, &b);
-      if (!warp_wait(smem_u32(&dfull[set]), (sg >> 1) & 1, s_abort)) break;
-      tc_fence_after();
       const int n = static_cast<int>(tile) * kTileRows + r;
       const float mul = __half2float(__ushort_as_half(p.scales[n]));
       const int c_lo = range_owner(tile * KS, total, G);
       const int c_hi = range_owner(tile * KS + KS - 1, total, G);
       const bool split = c_lo != c_hi;
-      const int which = (tile == tile_first) ? 0 : 1;   // this CTA's first or last segment
-      float* part = p.partials + static_cast<long long>(2 * c + which) * NCOL * 128;
-      for (int c0 = 0; c0 < mcount; c0 += 8) {
+      const bool finisher = (c == c_lo);
+      float pre[NCOL];
+#pragma unroll
+      for (int j = 0; j < NCOL; ++j) pre[j] = 0.0f;
+      if (split && finisher) {
+        // the other contributors' partials, summed in CTA order
+        if (!wait_counter(&p.counters[c_lo], 4u * static_cast<unsigned int>(c_hi - c_lo), s_abort)) break;
+        for (int cc = c_lo + 1; cc <= c_hi; ++cc) {
+          const float* src = p.partials + static_cast<long long>(cc) * NCOL * 128 + r;
+#pragma unroll
+          for (int j = 0; j < NCOL; ++j)
+            if (j < mcount) pre[j] += __ldcg(src + j * 128);
+        }
+        // Reset the counter for the next launch once all four warps have seen
+        // it complete (a CTA finishes at most one split tile: one meeting).
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&epi[0]));
+        if (quad == 0 && warp_wait(smem_u32(&epi[0]), 0, s_abort) && lane == 0) p.counters[c_lo] = 0u;
+      }
+      if (!warp_wait(smem_u32(&dfull[set]), (sg >> 1) & 1, s_abort)) break;
+      tc_fence_after();
+      float* part = p.partials + static_cast<long long>(c) * NCOL * 128 + r;
+#pragma unroll
+      for (int ch = 0; ch < NCOL / 8; ++ch) {
+        const int c0 = ch * 8;
+        if (c0 >= mcount) break;
         float acc[8];
 #pragma unroll
         for (int jj = 0; jj < 8; ++jj) acc[jj] = 0.0f;
@@ -317,59 +345,25 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 #pragma unroll
           for (int jj = 0; jj < 8; ++jj) acc[jj] += __uint_as_float(v[jj]);
         }
-        if (split) {
+        if (split && !finisher) {
 #pragma unroll
-          for (int jj = 0; jj < 8; ++jj) __stcg(part + (c0 + jj) * 128 + r, acc[jj]);
+          for (int jj = 0; jj < 8; ++jj) __stcg(part + (c0 + jj) * 128, acc[jj]);
         } else {
 #pragma unroll
-          for (int jj = 0; jj < 8; ++jj)
+          for (int jj = 0; jj < 8; ++jj) {
+            const float v = pre[c0 + jj] + acc[jj];
             if (c0 + jj < mcount)
-              p.y[static_cast<long long>(c0 + jj) * p.N + n] = __half_as_ushort(__float2half_rn(acc[jj] * mul));
+              p.y[static_cast<long long>(c0 + jj) * p.N + n] = __half_as_ushort(__float2half_rn(v * mul));
+          }
         }
       }
       // accumulators read: the set may be reused two segments on
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&dempty[set]));
-      if (split) {
-        // Publish this CTA's partial (release) and count arrivals; the last
-        // CTA of the tile (acquire) sums every partial in CTA order.  The
-        // warps meet on an mbarrier with a bounded wait.
-        const uint32_t eb = smem_u32(&epi[which]);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(eb);
-        if (!warp_wait(eb, 0, s_abort)) break;
-        if (leader) {
-          fence_acq_rel_gpu();
-          const unsigned int prev = atomicAdd(&p.counters[c_lo], 1u);
-          fence_acq_rel_gpu();
-          s_last[which] = (prev == static_cast<unsigned int>(c_hi - c_lo)) ? 1 : 0;
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(eb);
-        if (!warp_wait(eb, 1, s_abort)) break;
-        if (s_last[which]) {
-          for (int c0 = 0; c0 < mcount; c0 += 8) {
-            float acc[8];
-#pragma unroll
-            for (int jj = 0; jj < 8; ++jj) acc[jj] = 0.0f;
-            for (int cc = c_lo; cc <= c_hi; ++cc) {
-              const float* src = p.partials +
-                                 static_cast<long long>(partial_slot(cc, tile, total, G, KS)) * NCOL * 128 +
-                                 c0 * 128 + r;
-              float v[8];
-#pragma unroll
-              for (int jj = 0; jj < 8; ++jj) v[jj] = __ldcg(src + jj * 128);
-#pragma unroll
-              for (int jj = 0; jj < 8; ++jj) acc[jj] += v[jj];
-            }
-#pragma unroll
-            for (int jj = 0; jj < 8; ++jj)
-              if (c0 + jj < mcount)
-                p.y[static_cast<long long>(c0 + jj) * p.N + n] = __half_as_ushort(__float2half_rn(acc[jj] * mul));
-          }
-          if (leader) p.counters[c_lo] = 0u;
-        }
+      if (split && !finisher) {
+        __syncwarp();                        // the warp's partial rows are written
+        if (lane == 0) red_release_add(&p.counters[c_lo], 1u);
       }
     }
   }
