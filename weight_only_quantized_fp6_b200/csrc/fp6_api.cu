@@ -347,13 +347,29 @@ fp6_status fp6_linear(const uint16_t* x, const void* packed, const uint16_t* sca
   if (!encode) return FP6_ERR_CUDA;
   CUtensorMap map;
   std::memset(&map, 0, sizeof(map));
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * sizeof(uint16_t)};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(fp6::kTileCols), static_cast<cuuint32_t>(pl.ncol)};
-  const cuuint32_t estr[2] = {1, 1};
-  CUresult cr = encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t*>(x), dims, strides, box, estr,
-                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult cr;
+  if (pl.ncol <= 32) {
+    // decode kernel: x as [K/64][M][64] (column tile, row, column), one box of
+    // T column tiles x NCOL rows per pipeline step; rows >= M read as zero
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(fp6::kTileCols), static_cast<cuuint64_t>(M),
+                                static_cast<cuuint64_t>(K / fp6::kTileCols)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K) * sizeof(uint16_t),
+                                   static_cast<cuuint64_t>(fp6::kTileCols) * sizeof(uint16_t)};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(fp6::kTileCols), static_cast<cuuint32_t>(pl.ncol),
+                               static_cast<cuuint32_t>(pl.T)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    cr = encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<uint16_t*>(x), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  } else {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * sizeof(uint16_t)};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(fp6::kTileCols), static_cast<cuuint32_t>(pl.ncol)};
+    const cuuint32_t estr[2] = {1, 1};
+    cr = encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t*>(x), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  }
   if (cr != CUDA_SUCCESS) return FP6_ERR_CUDA;
 
   switch (pl.ncol) {

@@ -4,7 +4,7 @@
 // Same product and the same work split as fp6_linear_kernel (fp6_linear.cuh):
 // y[M,N] = x[M,K] . (scale (.) decode(W[N,K]))^T, fp32 accumulation, fp16 out,
 // persistent CTAs over equal ranges of (row tile, step) iterations, split
-// tiles finished by their last-arriving CTA in CTA order.  What differs is the
+// tiles finished, in CTA order, by the CTA holding their first steps.  What differs is the
 // pipeline, shaped for the memory-bound regime where the tensor core is nearly
 // idle and the integer pipe (the FP6 -> FP16 splice) and synchronisation
 // latency are what remain:
@@ -22,11 +22,15 @@
 //   warps 12..15  epilogue warpgroup: per segment, the three group
 //                 accumulators summed in group order, * scale, fp16
 //                 store or split-K partial and fix-up.  Accumulators are double
-//                 buffered across segments.
+//                 buffered across segments where TMEM has room (16 token
+//                 columns), single buffered otherwise.
 //   warp 16       weight producer: one bulk copy of T packed tiles per step.
-//   warp 17       activation producer: T TMA tile copies per step (NCOL rows
-//                 x 64 columns, 128-byte swizzle, rows at or beyond M filled
-//                 with zeros by the copy) into an smem ring.  Completion is
+//   warp 17       activation producer: one TMA box per step (T column tiles
+//                 of NCOL rows x 64 columns, 128-byte swizzle, rows at or
+//                 beyond M filled with zeros by the copy) into an smem ring.
+//                 One copy per step, not one per tile: the copies of one
+//                 issuing warp are served one after another, about 0.3 us
+//                 each, which is as long as a step takes.  Completion is
 //                 counted in bytes on each stage's barrier, so a stage is ready
 //                 as soon as its own copies land, whatever was issued after.
 //
@@ -57,16 +61,18 @@ constexpr int kDecThreads = 32 * (kDecXProdWarp + 1);      // 576
 template <int NCOL>
 struct DecodeShape {
   static_assert(NCOL == 16 || NCOL == 32, "decode variants: 16 or 32 token columns");
-  static constexpr int kTMax = (NCOL == 16) ? 2 : 1;        // tiles per step, at most
+  static constexpr int kTMax = 2;                           // tiles per step, at most
   static constexpr int kXTile = NCOL * 128;                 // NCOL rows x 64 fp16, 128-byte swizzled
   static constexpr int kXStage = kTMax * kXTile;
   static constexpr int kWStage = kTMax * kTileBytes;
-  static constexpr int kRX = 9;                             // x stages
-  static constexpr int kSW = (NCOL == 16) ? 15 : 27;        // weight stages
+  static constexpr int kRX = (NCOL == 16) ? 9 : 6;          // x stages
+  static constexpr int kSW = (NCOL == 16) ? 15 : 12;        // weight stages
   static constexpr int kSlots = 2 * kDecGroups;             // TMEM slots: two per group
   static constexpr int kSlotCols = kTMax * 32;
   static constexpr int kDCol = kSlots * kSlotCols;          // accumulators after the slots
-  static constexpr int kAccCols = 2 * kDecGroups * NCOL;    // [set][group][NCOL]
+  // accumulator sets: two (segments alternate) when they fit in TMEM
+  static constexpr int kSets = (kDCol + 2 * kDecGroups * NCOL <= static_cast<int>(kTmemCols)) ? 2 : 1;
+  static constexpr int kAccCols = kSets * kDecGroups * NCOL;  // [set][group][NCOL]
   static constexpr int kWOff = kRX * kXStage;
   static constexpr int kBarOff = kWOff + kSW * kWStage;
   // wfull, wempty [SW]; xfull, xempty [RX]; slot free [6]; dfull, dempty [2]; epi [2]; done
@@ -196,8 +202,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       if (lane == 0) {
         const uint32_t fb = smem_u32(&xfull[s]);
         mbar_arrive_expect_tx(fb, bytes);
-        for (int t = 0; t < T; ++t)
-          tma_load_2d(smem_u32(smem + s * S::kXStage + t * S::kXTile), &tmap_x, fb, (ks * T + t) * kTileCols, 0, pol);
+        tma_load_3d(smem_u32(smem + s * S::kXStage), &tmap_x, fb, 0, 0, ks * T, pol);
       }
       __syncwarp();
       ++issued;
@@ -218,11 +223,12 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     for (int sg = 0; sg < nseg; ++sg) {
       int a, b;
       segment_range(sg, tile_first, s0, KS, n_local, &a, &b);
-      const int set = sg & 1;
+      const int set = sg % S::kSets;
       const uint32_t d_tmem = tmem + S::kDCol + (set * kDecGroups + g) * NCOL;
-      // The accumulators of this set were last used two segments ago: the
+      // The accumulators of this set were last used kSets segments ago: the
       // epilogue must have read them before the first MMA or arrival.
-      if (issuer && sg >= 2) ok = warp_wait(smem_u32(&dempty[set]), ((sg >> 1) - 1) & 1, s_abort) && ok;
+      if (issuer && sg >= S::kSets)
+        ok = warp_wait(smem_u32(&dempty[set]), ((sg / S::kSets) - 1) & 1, s_abort) && ok;
       bool first = true;
       for (int li = group_first(g, a); li <= b; li += kDecGroups, ++j) {
         const int sw = li % kSW;
@@ -299,7 +305,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     const int mcount = min(NCOL, p.M);
     for (int sg = 0; sg < nseg; ++sg) {
       const long long tile = tile_first + sg;
-      const int set = sg & 1;
+      const int set = sg % S::kSets;
       int a, b;
       segment_range(sg, tile_first, s0, KS, n_local, &a, &b);
       const int n = static_cast<int>(tile) * kTileRows + r;
@@ -326,7 +332,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         if (lane == 0) mbar_arrive(smem_u32(&epi[0]));
         if (quad == 0 && warp_wait(smem_u32(&epi[0]), 0, s_abort) && lane == 0) p.counters[c_lo] = 0u;
       }
-      if (!warp_wait(smem_u32(&dfull[set]), (sg >> 1) & 1, s_abort)) break;
+      if (!warp_wait(smem_u32(&dfull[set]), (sg / S::kSets) & 1, s_abort)) break;
       tc_fence_after();
       float* part = p.partials + static_cast<long long>(c) * NCOL * 128 + r;
 #pragma unroll
@@ -357,7 +363,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
           }
         }
       }
-      // accumulators read: the set may be reused two segments on
+      // accumulators read: the set may be reused kSets segments on
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&dempty[set]));
