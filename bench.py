@@ -47,7 +47,7 @@ def algo_bytes(M, N, K):
     return 0.75 * N * K + 2 * N + 2 * M * K
 
 
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "fp6_linear_kernel_llama70b_o_proj_decode.md")
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "fp6_linear_decode_kernel_llama70b_o_proj_decode.md")
 
 
 def kernel_source_hash() -> str:
@@ -102,7 +102,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "20"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
         except (OSError, ValueError):
@@ -184,9 +184,9 @@ def oracle_workload(rows: int):
     return codes, scales, xs
 
 
-def time_oracle(rows: int, threads: int, reps: int = 1):
+def time_oracle(rows: int, threads: int, reps: int = 1, workload=None):
     import oracle
-    codes, scales, xs = oracle_workload(rows)
+    codes, scales, xs = workload if workload is not None else oracle_workload(rows)
     t0 = time.perf_counter()
     for _ in range(reps):
         for M in MS:
@@ -196,12 +196,17 @@ def time_oracle(rows: int, threads: int, reps: int = 1):
     return gbs, dt
 
 
-def cpu_baseline():
+def cpu_baseline(target_s: float = 10.0):
+    """The oracle on all host cores, on whole steps of the workload, repeated
+    until about `target_s` seconds of CPU work have been timed."""
     threads = os.cpu_count() or 1
-    rows = N_DIM  # the whole layer: a few seconds of all-core CPU work
-    gbs, dt = time_oracle(rows, threads)
+    rows = N_DIM  # the whole layer
+    work = oracle_workload(rows)
+    _, dt1 = time_oracle(rows, threads, workload=work)
+    reps = max(1, int(math.ceil(target_s / max(dt1, 1e-3))))
+    gbs, dt = time_oracle(rows, threads, reps=reps, workload=work)
     return {"value": round(gbs, 4), "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": f"one full step (N={N_DIM}, K={K_DIM}, M={MS}) on {threads} threads, {dt:.2f} s"}
+            "sample": f"{reps} full steps (N={N_DIM}, K={K_DIM}, M={MS}) on {threads} threads, {dt:.2f} s"}
 
 
 def run_reference(args, world, rank):
@@ -399,7 +404,7 @@ def run_fp6(args, world, rank, local):
                                           f"(algorithmic {algo_bytes(prof['M'], N_DIM, K_DIM):.0f} B)")
                          if prof else "no ncu capture of this kernel source",
                          "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs)",
-                         "kernel": "fp6_linear_kernel<16>"},
+                         "kernel": "fp6_linear_decode_kernel<16>"},
             "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": launches,
