@@ -102,7 +102,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "20"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
         except (OSError, ValueError):
@@ -112,7 +112,11 @@ class ClockSampler:
         for ln in self.proc.stdout:
             self.lines.append(ln.strip())
 
-    def stop(self):
+    def mark(self) -> int:
+        """Number of samples so far; stop(since=mark()) keeps only later ones."""
+        return len(self.lines)
+
+    def stop(self, since: int = 0):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
@@ -122,7 +126,7 @@ class ClockSampler:
             self.proc.kill()
         sm, smax, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for ln in self.lines[since:]:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 9:
                 continue
@@ -196,7 +200,7 @@ def time_oracle(rows: int, threads: int, reps: int = 1, workload=None):
     return gbs, dt
 
 
-def cpu_baseline(target_s: float = 10.0):
+def cpu_baseline(target_s: float = 15.0):
     """The oracle on all host cores, on whole steps of the workload, repeated
     until about `target_s` seconds of CPU work have been timed."""
     threads = os.cpu_count() or 1
@@ -237,6 +241,84 @@ def run_reference(args, world, rank):
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+# ---- context measurements outside the timed region ---------------------------------
+
+PREFILL_SHAPES = [(28672, 8192), (8192, 28672)]   # Llama-70B-shaped gate/up and down halves
+PREFILL_MS = [256, 1024, 4096]
+
+
+def _time_us(fn, stream, reps=10):
+    """Average device time of fn() over `reps` calls on `stream` (after one warm-up call)."""
+    import torch
+    with torch.cuda.stream(stream):
+        fn()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) * 1e3 / reps
+
+
+def measure_prefill_and_ablation(dev, stream, peaks, packs, scales, xs):
+    """Compute-bound prefill sizes (TFLOP/s against the measured dense bf16/fp16
+    peak) and the two-kernel comparison of the pages (separate dequant kernel,
+    then a cuBLAS fp16 GEMM) next to the fused kernel and a plain fp16 GEMM
+    (cuBLAS W16A16).  cuBLAS appears only here, as context."""
+    import torch
+
+    import weight_only_quantized_fp6_b200 as fp6
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(5000)
+    prefill, ablation = [], []
+    ws = fp6.Workspace(dev)
+    for (N, K) in PREFILL_SHAPES:
+        W = torch.randn(N, K, device=dev, generator=gen) * 0.02
+        layer = fp6.FP6Linear.from_float(W)
+        del W
+        W16 = fp6.dequant(layer.packed, layer.scales, N, K)
+        for M in PREFILL_MS:
+            x = torch.randn(M, K, device=dev, generator=gen).half()
+            y = torch.empty((M, N), dtype=torch.float16, device=dev)
+            ws.get(fp6.workspace_bytes(M, N, K))
+            t = _time_us(lambda: fp6.linear(x, layer.packed, layer.scales, N, K, out=y, workspace=ws), stream)
+            t16 = _time_us(lambda: torch.matmul(x, W16.t()), stream)
+            t2 = _time_us(lambda: torch.matmul(x, fp6.dequant(layer.packed, layer.scales, N, K).t()), stream)
+            fl = 2.0 * M * N * K
+            prefill.append({"N": N, "K": K, "M": M, "us": round(t, 2), "tflops": round(fl / t / 1e6, 1),
+                            "frac_of_peak": round(fl / t / 1e6 / peaks["bf16_tflops"], 4)})
+            ablation.append({"N": N, "K": K, "M": M, "fused_us": round(t, 2), "dequant_then_gemm_us": round(t2, 2),
+                             "cublas_w16a16_us": round(t16, 2)})
+        del layer, W16
+    # decode shape: rotate the packed copies (and the fp16 copies, 134 MB each) past L2
+    N, K = N_DIM, K_DIM
+    W16s = [fp6.dequant(packs[i], scales, N, K) for i in range(2)]
+    for M in (1, 16):
+        x = xs[M]
+        cnt = [0]
+
+        def fused():
+            cnt[0] += 1
+            fp6.linear(x, packs[cnt[0] % len(packs)], scales, N, K, out=y16)
+
+        def two_kernel():
+            cnt[0] += 1
+            torch.matmul(x, fp6.dequant(packs[cnt[0] % len(packs)], scales, N, K).t())
+
+        def w16():
+            cnt[0] += 1
+            torch.matmul(x, W16s[cnt[0] % 2].t())
+
+        y16 = torch.empty((M, N), dtype=torch.float16, device=dev)
+        ablation.append({"N": N, "K": K, "M": M, "fused_us": round(_time_us(fused, stream, 22), 2),
+                         "dequant_then_gemm_us": round(_time_us(two_kernel, stream, 22), 2),
+                         "cublas_w16a16_us": round(_time_us(w16, stream, 22), 2)})
+    del W16s
+    return prefill, ablation
 
 
 # ---- the GPU arm -------------------------------------------------------------------
@@ -296,7 +378,8 @@ def run_fp6(args, world, rank, local):
 
     sampler = ClockSampler(local)
     sampler.start()
-    time.sleep(0.3)
+    time.sleep(0.5)                          # nvidia-smi start-up
+    since = sampler.mark()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     barrier(world)
@@ -309,7 +392,20 @@ def run_fp6(args, world, rank, local):
     torch.cuda.synchronize()
     barrier(world)
     elapsed_ms = t_start.elapsed_time(t_end)
-    clocks = sampler.stop()
+    # The timed region lasts milliseconds, less than the sampling period: keep
+    # replaying the same step (untimed) for 0.5 s so the clock record covers
+    # this load.
+    t_soak = time.perf_counter()
+    with torch.cuda.stream(stream):
+        s = 0
+        while time.perf_counter() - t_soak < 0.5:
+            step(s)
+            s += 1
+            if s % 64 == 0:
+                stream.synchronize()
+    torch.cuda.synchronize()
+    clocks = sampler.stop(since)
+    clocks["window"] = "timed region + 0.5 s of the same graph replays right after it"
 
     elapsed_max = max_over_ranks(elapsed_ms, world)
     launches = args.steps * len(MS)
@@ -375,6 +471,9 @@ def run_fp6(args, world, rank, local):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
     e2e_value = world * e2e_steps * len(MS) * wbytes(N_DIM, K_DIM) / (e2e_ms / 1e3) / 1e9
 
+    prefill, ablation = (measure_prefill_and_ablation(dev, stream, peaks, packs, scales, xs)
+                         if rank == 0 and not args.no_extra else (None, None))
+
     ok = fp6.device_status(dev)
     if ok != 0:
         raise SystemExit(f"device error word set: {ok}")
@@ -410,6 +509,14 @@ def run_fp6(args, world, rank, local):
             "gpu_launches": launches,
             "clocks": clocks,
         }
+        if prefill is not None:
+            line["prefill"] = {"metric": "TFLOP/s, fused kernel, M >= 256 (tensor-bound sizes)",
+                               "peak_tflops": peaks["bf16_tflops"],
+                               "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json bf16_tflops; fp16 runs at "
+                                              f"the bf16 rate)", "runs": prefill}
+            line["ablation"] = {"note": "separate dequant kernel + cuBLAS fp16 GEMM, and cuBLAS fp16 GEMM on "
+                                        "the dequantized weights (W16A16), against the fused kernel; "
+                                        "per launch, microseconds", "runs": ablation}
         if cpu is not None:
             line["cpu_baseline"] = cpu
         print(json.dumps(line), flush=True)
@@ -422,6 +529,8 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["fp6", "reference"], default="fp6")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the prefill and two-kernel context measurements (outside the timed region)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
