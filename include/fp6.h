@@ -142,6 +142,17 @@ fp6_status fp6_linear(const uint16_t *x, const void *packed, const uint16_t *sca
 fp6_status fp6_get_device_status(struct CUstream_st *stream);
 
 /*
+ * fp6_selftest_wait_timeout -- failure-detection self-test; the FP6-LLM pages
+ * have no counterpart.  Enqueues a one-warp kernel that waits on an mbarrier
+ * nothing ever arrives on, through the same bounded wait the linear kernels
+ * use.  The wait gives up after its limit (about 2 s), sets the device error
+ * word and the kernel exits: the next fp6_get_device_status on the stream
+ * returns FP6_ERR_TIMEOUT (and clears the word), and the context stays usable.
+ * Returns FP6_ERR_CUDA if the launch fails, else FP6_OK.
+ */
+fp6_status fp6_selftest_wait_timeout(struct CUstream_st *stream);
+
+/*
  * fp6_linear_noalloc -- fp6_linear for callers that cannot allocate device
  * memory while the layer runs (for example a plugin inside an engine that owns
  * all device memory, or a latency-critical loop where cudaMalloc, which may

@@ -132,6 +132,8 @@ def linear(x, packed, scales, N: int, K: int, out=None, workspace: Workspace | N
     M, K2 = x.shape
     if K2 != K or scales.shape[0] != N:
         raise ValueError("shape mismatch between x, scales and (N, K)")
+    if N > 0 and K > 0 and packed.numel() < packed_bytes(N, K):
+        raise ValueError(f"packed holds {packed.numel()} bytes; an {N} x {K} weight needs {packed_bytes(N, K)}")
     if out is None:
         out = torch.empty((M, N), dtype=torch.float16, device=x.device)
     else:

@@ -14,6 +14,23 @@
 #include "fp6_linear.cuh"
 #include "fp6_linear_decode.cuh"
 
+namespace fp6 {
+// A wait that can never complete: the mbarrier expects one arrival that no
+// thread makes.  The bounded wait gives up after its time limit, raises the
+// device error word and returns; the kernel then exits normally.
+__global__ void wait_timeout_kernel() {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  warp_wait(smem_u32(&bar), 0, &abort_flag);
+}
+}  // namespace fp6
+
 namespace {
 
 using fp6::DecodeShape;
@@ -392,6 +409,11 @@ fp6_status fp6_get_device_status(cudaStream_t stream) {
     return FP6_ERR_CUDA;
   if (cudaStreamSynchronize(stream) != cudaSuccess) return FP6_ERR_CUDA;
   return (word & fp6::kErrTimeout) ? FP6_ERR_TIMEOUT : FP6_OK;
+}
+
+fp6_status fp6_selftest_wait_timeout(cudaStream_t stream) {
+  fp6::wait_timeout_kernel<<<1, 32, 0, stream>>>();
+  return cuda_status(cudaGetLastError());
 }
 
 // ---- allocation-free variant -------------------------------------------------
