@@ -523,17 +523,86 @@ def run_fp6(args, world, rank, local):
     return 0
 
 
+def run_sweep(args):
+    """Every layer shape and M of the Llama-70B, OPT-30B and prefill configs:
+    per-launch time (a CUDA graph of launches rotating over enough packed-weight
+    copies that no launch finds its weights in L2), weight GB/s, TFLOP/s and the
+    fraction of the roofline max(2MNK / P_tensor, (0.75NK + 2N + 2MK) / BW_hbm).
+    Weights and activations come from torch's seeded CUDA generator: the
+    times do not depend on the values (parity is the tests' job)."""
+    import torch
+
+    import weight_only_quantized_fp6_b200 as fp6
+    from weight_only_quantized_fp6_b200 import inputs
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    l2 = getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 126 * 1024 * 1024)
+    peaks = read_peaks()
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(6000)
+    stream = torch.cuda.Stream(device=dev)
+    ws = fp6.Workspace(dev)
+    rows = []
+    for cfg in (2, 3, 4, 5):
+        spec = inputs.CONFIGS[cfg]
+        for lname, (N, K) in spec["layers"].items():
+            W = torch.randn(N, K, device=dev, generator=gen) * 0.02
+            layer = fp6.FP6Linear.from_float(W)
+            del W
+            copies = max(1, min(8, math.ceil(4 * l2 / wbytes(N, K))))
+            packs = [layer.packed] + [layer.packed.clone() for _ in range(copies - 1)]
+            for M in spec["M"]:
+                x = torch.randn(M, K, device=dev, generator=gen).half()
+                y = torch.empty((M, N), dtype=torch.float16, device=dev)
+                ws.get(fp6.workspace_bytes(M, N, K))
+                n_launch = max(2 * copies, 8)
+                with torch.cuda.stream(stream):
+                    fp6.linear(x, packs[0], layer.scales, N, K, out=y, workspace=ws)
+                    stream.synchronize()
+                    graph = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(graph, stream=stream):
+                        for i in range(n_launch):
+                            fp6.linear(x, packs[i % copies], layer.scales, N, K, out=y, workspace=ws)
+                    graph.replay()
+                    e0 = torch.cuda.Event(enable_timing=True)
+                    e1 = torch.cuda.Event(enable_timing=True)
+                    e0.record()
+                    for _ in range(3):
+                        graph.replay()
+                    e1.record()
+                torch.cuda.synchronize()
+                t = e0.elapsed_time(e1) * 1e-3 / (3 * n_launch)
+                del graph
+                t_tc = 2.0 * M * N * K / (peaks["bf16_tflops"] * 1e12)
+                t_hbm = algo_bytes(M, N, K) / (peaks["hbm_gbs"] * 1e9)
+                rows.append({"config": spec["name"], "layer": lname, "N": N, "K": K, "M": M,
+                             "us": round(t * 1e6, 2), "weight_gbs": round(wbytes(N, K) / t / 1e9, 1),
+                             "tflops": round(2.0 * M * N * K / t / 1e12, 1),
+                             "bound": "tensor" if t_tc > t_hbm else "hbm",
+                             "roofline_frac": round(max(t_tc, t_hbm) / t, 4)})
+                print(json.dumps(rows[-1]), file=sys.stderr, flush=True)
+            del layer, packs
+    if fp6.device_status(dev) != 0:
+        raise SystemExit("device error word set")
+    print(json.dumps({"sweep": rows, "peaks": peaks, "l2_bytes": l2}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["fp6", "reference"], default="fp6")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time every layer shape and M of the Llama-70B, OPT-30B and prefill configs (1 GPU)")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the prefill and two-kernel context measurements (outside the timed region)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.sweep:
+        return run_sweep(args)
     world, rank, local = dist_setup(args)
     try:
         if args.impl == "reference":

@@ -52,7 +52,7 @@ fp6_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FP6_OK : FP6_E
 // ---- per-device cached properties ------------------------------------------
 struct DeviceInfo {
   int sms = 0;
-  bool attrs_set[7] = {false, false, false, false, false, false, false};
+  bool attrs_set[8] = {false, false, false, false, false, false, false, false};
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -110,13 +110,14 @@ int pick_ncol(int64_t M) {
   return 256;
 }
 
-// Token tiles of up to 32 columns run the decode kernel (fp6_linear_decode.cuh),
-// wider ones the general kernel (fp6_linear.cuh).
+// One token tile of up to 64 columns runs the decode kernel
+// (fp6_linear_decode.cuh), wider or several token tiles the general kernel
+// (fp6_linear.cuh).
 int tmax_for(int ncol) {
   switch (ncol) {
     case 16: return DecodeShape<16>::kTMax;
     case 32: return DecodeShape<32>::kTMax;
-    case 64: return LinearShape<64>::kTMax;
+    case 64: return DecodeShape<64>::kTMax;
     case 128: return LinearShape<128>::kTMax;
     default: return LinearShape<256>::kTMax;
   }
@@ -126,7 +127,7 @@ int stages_for(int ncol) {
   switch (ncol) {
     case 16: return DecodeShape<16>::kSW;
     case 32: return DecodeShape<32>::kSW;
-    case 64: return LinearShape<64>::kSW;
+    case 64: return DecodeShape<64>::kSW;
     case 128: return LinearShape<128>::kSW;
     default: return LinearShape<256>::kSW;
   }
@@ -187,12 +188,12 @@ fp6_status launch_linear(const CUtensorMap& map, const fp6::LinearParams& prm, c
   return cuda_status(cudaGetLastError());
 }
 
-// The decode kernel (one token tile of at most 32 columns), launched the same way.
+// The decode kernel (one token tile of at most 64 columns), launched the same way.
 template <int NCOL>
 fp6_status launch_decode(const CUtensorMap& map, const fp6::LinearParams& prm, cudaStream_t stream, int dev) {
   auto kern = fp6::fp6_linear_decode_kernel<NCOL>;
   const int smem = DecodeShape<NCOL>::kSmemBytes;
-  const int idx = NCOL == 16 ? 5 : 6;
+  const int idx = NCOL == 16 ? 5 : NCOL == 32 ? 6 : 7;
   {
     std::lock_guard<std::mutex> lk(g_mu);
     if (!g_dev[dev].attrs_set[idx]) {
@@ -203,7 +204,7 @@ fp6_status launch_decode(const CUtensorMap& map, const fp6::LinearParams& prm, c
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned int>(prm.grid));
-  cfg.blockDim = dim3(static_cast<unsigned int>(fp6::kDecThreads));
+  cfg.blockDim = dim3(static_cast<unsigned int>(DecodeShape<NCOL>::kThreads));
   cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -364,35 +365,24 @@ fp6_status fp6_linear(const uint16_t* x, const void* packed, const uint16_t* sca
   if (!encode) return FP6_ERR_CUDA;
   CUtensorMap map;
   std::memset(&map, 0, sizeof(map));
-  CUresult cr;
-  if (pl.ncol <= 32) {
-    // decode kernel: x as [K/64][M][64] (column tile, row, column), one box of
-    // T column tiles x NCOL rows per pipeline step; rows >= M read as zero
-    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(fp6::kTileCols), static_cast<cuuint64_t>(M),
-                                static_cast<cuuint64_t>(K / fp6::kTileCols)};
-    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K) * sizeof(uint16_t),
-                                   static_cast<cuuint64_t>(fp6::kTileCols) * sizeof(uint16_t)};
-    const cuuint32_t box[3] = {static_cast<cuuint32_t>(fp6::kTileCols), static_cast<cuuint32_t>(pl.ncol),
-                               static_cast<cuuint32_t>(pl.T)};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    cr = encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<uint16_t*>(x), dims, strides, box, estr,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  } else {
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * sizeof(uint16_t)};
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(fp6::kTileCols), static_cast<cuuint32_t>(pl.ncol)};
-    const cuuint32_t estr[2] = {1, 1};
-    cr = encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t*>(x), dims, strides, box, estr,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  }
+  // x as [K/64][M][64] (column tile, row, column): one box of T column tiles x
+  // NCOL rows per pipeline step; rows >= M read as zero
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(fp6::kTileCols), static_cast<cuuint64_t>(M),
+                              static_cast<cuuint64_t>(K / fp6::kTileCols)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K) * sizeof(uint16_t),
+                                 static_cast<cuuint64_t>(fp6::kTileCols) * sizeof(uint16_t)};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(fp6::kTileCols), static_cast<cuuint32_t>(pl.ncol),
+                             static_cast<cuuint32_t>(pl.T)};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult cr = encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<uint16_t*>(x), dims, strides, box,
+                             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (cr != CUDA_SUCCESS) return FP6_ERR_CUDA;
 
   switch (pl.ncol) {
     case 16: return launch_decode<16>(map, prm, stream, dev);
     case 32: return launch_decode<32>(map, prm, stream, dev);
-    case 64: return launch_linear<64>(map, prm, stream, dev);
+    case 64: return launch_decode<64>(map, prm, stream, dev);
     case 128: return launch_linear<128>(map, prm, stream, dev);
     default: return launch_linear<256>(map, prm, stream, dev);
   }

@@ -13,10 +13,8 @@
 //
 //   warp 20       weight producer: one bulk copy of the step's T packed tiles
 //                 (contiguous, T * 6144 bytes) into a smem ring (SW stages);
-//   warp 21       activation producer into a ring of RX stages: for one token
-//                 tile (M <= NCOL <= 64) 16-byte cp.async copies of the M valid
-//                 rows (x stays off the TMA engine, which the weight stream keeps
-//                 busy); otherwise T TMA tile copies (NCOL rows x 64, 128-byte
+//   warp 21       activation producer into a ring of RX stages: one TMA box
+//                 per step (T column tiles of NCOL rows x 64 columns, 128-byte
 //                 swizzle, rows beyond M zero-filled);
 //   warps 8..19   three dequant warpgroups taking every third step: each thread
 //                 owns one weight row (its TMEM lane), reads its 48 packed bytes
@@ -103,7 +101,7 @@ struct LinearShape {
 };
 
 struct LinearParams {
-  const uint16_t* x;     // [M,K] fp16 (read directly by the decode kernel; the prefill kernel uses TMA)
+  const uint16_t* x;     // [M,K] fp16 (the kernels read it through the tensor map)
   const uint8_t* packed;
   const uint16_t* scales;
   uint16_t* y;
@@ -276,70 +274,23 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
   } else if (warp == kXProdWarp) {
     // ---------------- activation producer ----------------
     grid_dependency_wait();                  // x is written by earlier work in the stream
-    if constexpr (NCOL <= 64) {
-      // One token tile (M <= NCOL): LSU copies keep x off the TMA engine,
-      // which the weight stream keeps busy.  Rows at or beyond M are never
-      // loaded, so every stage is zeroed once; each step copies the M valid
-      // rows of its T x tiles in 16-byte chunks straight into the
-      // 128-byte-swizzled layout (chunk ch of row r at (ch ^ (r % 8)) * 16).
-      for (int i = lane; i < kRX * S::kXStage / 16; i += 32)
-        *reinterpret_cast<uint4*>(smem + i * 16) = make_uint4(0u, 0u, 0u, 0u);
-      __syncwarp();
-      constexpr int kDepth = (kRX - 2 < 3) ? kRX - 2 : 3;   // steps in flight besides the newest
-      const int chunks_per_row = T * 8;
-      const int chunks = p.M * chunks_per_row;
-      int ks = static_cast<int>(s0 - tile_first * KS);
-      int signalled = 0;
-      int issued = 0;
-      for (int li = 0; li < n_local; ++li, ks = (ks + 1 == KS) ? 0 : ks + 1) {
-        const int s = li % kRX;
-        if (li >= kRX && !warp_wait(smem_u32(&xempty[s]), ((li / kRX) - 1) & 1, s_abort)) break;
-        uint8_t* stage = smem + s * S::kXStage;
-        const uint16_t* src0 = p.x + static_cast<long long>(ks) * T * kTileCols;
-        for (int idx = lane; idx < chunks; idx += 32) {
-          const int r = idx / chunks_per_row;
-          const int rem = idx - r * chunks_per_row;
-          const int t = rem >> 3, ch = rem & 7;
-          cp_async_16(smem_u32(stage + t * S::kXTile + r * 128 + ((ch ^ (r & 7)) << 4)),
-                      src0 + static_cast<long long>(r) * p.K + t * kTileCols + ch * 8);
-        }
-        cp_async_commit();
-        ++issued;
-        if (issued - signalled > kDepth) {
-          // the oldest step's copies have landed: make them visible to the tensor core
-          cp_async_wait<kDepth>();
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(&xfull[signalled % kRX]));
-          ++signalled;
-        }
+    const uint64_t pol = policy_evict_last();
+    StepCursor cur(s0, KS, MT);
+    const uint32_t bytes = static_cast<uint32_t>(T) * S::kXTile;
+    int issued = 0;
+    for (int li = 0; li < n_local; ++li, cur.next()) {
+      const int s = li % kRX;
+      if (li >= kRX && !warp_wait(smem_u32(&xempty[s]), ((li / kRX) - 1) & 1, s_abort)) break;
+      if (lane == 0) {
+        const uint32_t fb = smem_u32(&xfull[s]);
+        mbar_arrive_expect_tx(fb, bytes);
+        tma_load_3d(smem_u32(smem + s * S::kXStage), &tmap_x, fb, 0, cur.mt * NCOL, cur.ks * T, pol);
       }
-      cp_async_wait<0>();
-      fence_proxy_async_smem();
       __syncwarp();
-      for (; signalled < issued; ++signalled)
-        if (lane == 0) mbar_arrive(smem_u32(&xfull[signalled % kRX]));
-    } else {
-      const uint64_t pol = policy_evict_last();
-      StepCursor cur(s0, KS, MT);
-      const uint32_t bytes = static_cast<uint32_t>(T) * S::kXTile;
-      int issued = 0;
-      for (int li = 0; li < n_local; ++li, cur.next()) {
-        const int s = li % kRX;
-        if (li >= kRX && !warp_wait(smem_u32(&xempty[s]), ((li / kRX) - 1) & 1, s_abort)) break;
-        if (lane == 0) {
-          const uint32_t fb = smem_u32(&xfull[s]);
-          mbar_arrive_expect_tx(fb, bytes);
-          for (int t = 0; t < T; ++t)
-            tma_load_2d(smem_u32(smem + s * S::kXStage + t * S::kXTile), &tmap_x, fb,
-                        (cur.ks * T + t) * kTileCols, cur.mt * NCOL, pol);
-        }
-        __syncwarp();
-        ++issued;
-      }
-      for (int li = issued > kRX ? issued - kRX : 0; li < issued; ++li)
-        warp_wait(smem_u32(&xfull[li % kRX]), (li / kRX) & 1, s_never);
+      ++issued;
     }
+    for (int li = issued > kRX ? issued - kRX : 0; li < issued; ++li)
+      warp_wait(smem_u32(&xfull[li % kRX]), (li / kRX) & 1, s_never);
   } else if (warp < kISS) {
     // ---------------- MMA issuer `warp`: k-slice [warp*4/kISS, (warp+1)*4/kISS) of every tile ----------------
     constexpr uint32_t idesc = idesc_f16_f32(128, NCOL);

@@ -9,8 +9,9 @@
 // idle and the integer pipe (the FP6 -> FP16 splice) and synchronisation
 // latency are what remain:
 //
-//   warps 0..11   three dequant groups of four warps (one per TMEM lane
-//                 quadrant), taking every third step.  A group splices its
+//   warps 0..4G-1 G dequant groups of four warps (one per TMEM lane
+//                 quadrant), taking every G-th step (G = 3; G = 2 for 64 token
+//                 columns, where three groups' TMEM would not fit).  A group splices its
 //                 step's T tiles into one of its own two TMEM slots, meets on a
 //                 hardware named barrier, and one warp of the group (quadrant
 //                 g, so the three groups issue from three different SM
@@ -19,13 +20,13 @@
 //                 step's dequant-to-MMA path is one barrier, and the slot it
 //                 refills next was released by the group's own commit two
 //                 steps earlier, long done.
-//   warps 12..15  epilogue warpgroup: per segment, the three group
+//   warps 4G..    epilogue warpgroup (four warps): per segment, the G group
 //                 accumulators summed in group order, * scale, fp16
 //                 store or split-K partial and fix-up.  Accumulators are double
 //                 buffered across segments where TMEM has room (16 token
 //                 columns), single buffered otherwise.
-//   warp 16       weight producer: one bulk copy of T packed tiles per step.
-//   warp 17       activation producer: one TMA box per step (T column tiles
+//   next warp     weight producer: one bulk copy of T packed tiles per step.
+//   last warp     activation producer: one TMA box per step (T column tiles
 //                 of NCOL rows x 64 columns, 128-byte swizzle, rows at or
 //                 beyond M filled with zeros by the copy) into an smem ring.
 //                 One copy per step, not one per tile: the copies of one
@@ -35,7 +36,7 @@
 //                 as soon as its own copies land, whatever was issued after.
 //
 // Ring ownership keeps every mbarrier's waits in phase order: weight stages
-// (SW) and x stages (RX) are multiples of three, so each stage is always used
+// (SW) and x stages (RX) are multiples of G, so each stage is always used
 // by the same group; TMEM slots and accumulators belong to one group.
 //
 // Named barriers cannot time out, so the group loops never leave early: a
@@ -52,34 +53,36 @@
 
 namespace fp6 {
 
-constexpr int kDecGroups = 3;
-constexpr int kDecEpiWarp = 12;                            // warps 12..15
-constexpr int kDecWProdWarp = 16;
-constexpr int kDecXProdWarp = 17;
-constexpr int kDecThreads = 32 * (kDecXProdWarp + 1);      // 576
 
 template <int NCOL>
 struct DecodeShape {
-  static_assert(NCOL == 16 || NCOL == 32, "decode variants: 16 or 32 token columns");
+  static_assert(NCOL == 16 || NCOL == 32 || NCOL == 64, "decode variants: 16, 32 or 64 token columns");
+  // dequant groups: three, or two where three groups' TMEM slots and
+  // accumulators would not fit in the 512 columns (64 token columns)
+  static constexpr int kGroups = (NCOL == 64) ? 2 : 3;
+  static constexpr int kEpiWarp = 4 * kGroups;              // four epilogue warps
+  static constexpr int kWProdWarp = kEpiWarp + 4;
+  static constexpr int kXProdWarp = kWProdWarp + 1;
+  static constexpr int kThreads = 32 * (kXProdWarp + 1);   // 576 (three groups) or 448
   static constexpr int kTMax = 2;                           // tiles per step, at most
   static constexpr int kXTile = NCOL * 128;                 // NCOL rows x 64 fp16, 128-byte swizzled
   static constexpr int kXStage = kTMax * kXTile;
   static constexpr int kWStage = kTMax * kTileBytes;
-  static constexpr int kRX = (NCOL == 16) ? 9 : 6;          // x stages
-  static constexpr int kSW = (NCOL == 16) ? 15 : 12;        // weight stages
-  static constexpr int kSlots = 2 * kDecGroups;             // TMEM slots: two per group
+  static constexpr int kRX = (NCOL == 16) ? 9 : (NCOL == 32) ? 6 : 4;   // x stages
+  static constexpr int kSW = (NCOL == 16) ? 15 : 12;                    // weight stages
+  static constexpr int kSlots = 2 * kGroups;               // TMEM slots: two per group
   static constexpr int kSlotCols = kTMax * 32;
   static constexpr int kDCol = kSlots * kSlotCols;          // accumulators after the slots
   // accumulator sets: two (segments alternate) when they fit in TMEM
-  static constexpr int kSets = (kDCol + 2 * kDecGroups * NCOL <= static_cast<int>(kTmemCols)) ? 2 : 1;
-  static constexpr int kAccCols = kSets * kDecGroups * NCOL;  // [set][group][NCOL]
+  static constexpr int kSets = (kDCol + 2 * kGroups * NCOL <= static_cast<int>(kTmemCols)) ? 2 : 1;
+  static constexpr int kAccCols = kSets * kGroups * NCOL;   // [set][group][NCOL]
   static constexpr int kWOff = kRX * kXStage;
   static constexpr int kBarOff = kWOff + kSW * kWStage;
   // wfull, wempty [SW]; xfull, xempty [RX]; slot free [6]; dfull, dempty [2]; epi [2]; done
   static constexpr int kNumBars = 2 * kSW + 2 * kRX + kSlots + 2 + 2 + 2 + 1;
   static constexpr int kBarrierBytes = 1024;
   static constexpr int kSmemBytes = kBarOff + kBarrierBytes + 1024;  // + alignment slack
-  static_assert(kSW % kDecGroups == 0 && kRX % kDecGroups == 0, "stages owned by one group");
+  static_assert(kSW % kGroups == 0 && kRX % kGroups == 0, "stages owned by one group");
   static_assert(kDCol + kAccCols <= static_cast<int>(kTmemCols), "TMEM budget");
   static_assert(kXTile % 1024 == 0 && kTileBytes % 1024 == 0, "1024-byte aligned tiles");
   static_assert(kNumBars * 8 + 32 <= kBarrierBytes, "barrier area");
@@ -96,12 +99,12 @@ __device__ __forceinline__ void segment_range(int sg, long long tile_first, long
 }
 
 // First step of group g (steps li with li % 3 == g) at or after a.
-__device__ __forceinline__ int group_first(int g, int a) {
-  return a + ((g - a % kDecGroups) + kDecGroups) % kDecGroups;
+__device__ __forceinline__ int group_first(int g, int a, int groups) {
+  return a + ((g - a % groups) + groups) % groups;
 }
 
 template <int NCOL>
-__global__ void __launch_bounds__(kDecThreads, 1)
+__global__ void __launch_bounds__(DecodeShape<NCOL>::kThreads, 1)
     fp6_linear_decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const LinearParams p) {
   using S = DecodeShape<NCOL>;
   constexpr int kSW = S::kSW;
@@ -145,9 +148,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     const int bx = 2 * kSW, bs = bx + 2 * kRX, bd = bs + S::kSlots;
     uint32_t count = 1;                                       // wfull, xfull, xempty, slotfree
     if (b >= kSW && b < bx) count = 4;                        // wempty: the group's four warps
-    else if (b >= bd && b < bd + 2) count = kDecGroups;       // dfull: one arrival per group
+    else if (b >= bd && b < bd + 2) count = S::kGroups;       // dfull: one arrival per group
     else if (b >= bd + 2 && b < bd + 6) count = 4;            // dempty, epi: epilogue warps
-    else if (b == bd + 6) count = kDecGroups;                 // done: one commit per group
+    else if (b == bd + 6) count = S::kGroups;                 // done: one commit per group
     mbar_init(smem_u32(&bars[b]), count);
     fence_barrier_init();
   }
@@ -157,7 +160,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     *s_abort = 0;
     *s_never = 0;
   }
-  if (warp == kDecXProdWarp && lane == 0) prefetch_tensormap(&tmap_x);
+  if (warp == S::kXProdWarp && lane == 0) prefetch_tensormap(&tmap_x);
   if (warp == 0) {
     tmem_alloc(smem_u32(tmem_holder), kTmemCols);
     tmem_relinquish();
@@ -168,7 +171,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  if (warp == kDecWProdWarp) {
+  if (warp == S::kWProdWarp) {
     // ---------------- weight producer ----------------
     const uint64_t pol = policy_evict_first();
     StepCursor cur(s0, KS, 1);
@@ -189,7 +192,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     }
     for (int li = issued > kSW ? issued - kSW : 0; li < issued; ++li)
       warp_wait(smem_u32(&wfull[li % kSW]), (li / kSW) & 1, s_never);
-  } else if (warp == kDecXProdWarp) {
+  } else if (warp == S::kXProdWarp) {
     // ---------------- activation producer ----------------
     grid_dependency_wait();                  // x is written by earlier work in the stream
     const uint64_t pol = policy_evict_last();
@@ -210,7 +213,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     // Leave no copy in flight.
     for (int li = issued > kRX ? issued - kRX : 0; li < issued; ++li)
       warp_wait(smem_u32(&xfull[li % kRX]), (li / kRX) & 1, s_never);
-  } else if (warp < 4 * kDecGroups) {
+  } else if (warp < 4 * S::kGroups) {
     // ---------------- dequant groups, each issuing its own MMAs ----------------
     const int g = warp >> 2;
     const int quad = warp & 3;               // TMEM lanes 32*quad .. 32*quad+31
@@ -224,13 +227,13 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       int a, b;
       segment_range(sg, tile_first, s0, KS, n_local, &a, &b);
       const int set = sg % S::kSets;
-      const uint32_t d_tmem = tmem + S::kDCol + (set * kDecGroups + g) * NCOL;
+      const uint32_t d_tmem = tmem + S::kDCol + (set * S::kGroups + g) * NCOL;
       // The accumulators of this set were last used kSets segments ago: the
       // epilogue must have read them before the first MMA or arrival.
       if (issuer && sg >= S::kSets)
         ok = warp_wait(smem_u32(&dempty[set]), ((sg / S::kSets) - 1) & 1, s_abort) && ok;
       bool first = true;
-      for (int li = group_first(g, a); li <= b; li += kDecGroups, ++j) {
+      for (int li = group_first(g, a, S::kGroups); li <= b; li += S::kGroups, ++j) {
         const int sw = li % kSW;
         const int sx = li % kRX;
         const int slot = 2 * g + (j & 1);
@@ -288,7 +291,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       __syncwarp();
       warp_wait(smem_u32(done), 0, s_never);
     }
-  } else if (warp >= kDecEpiWarp && warp < kDecEpiWarp + 4) {
+  } else if (warp >= S::kEpiWarp && warp < S::kEpiWarp + 4) {
     // ---------------- epilogue warpgroup: segments in order ----------------
     // A split row tile is finished by its first CTA c_lo, which reaches the
     // tile at the end of its range; every later contributor reaches it at the
@@ -342,11 +345,11 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         float acc[8];
 #pragma unroll
         for (int jj = 0; jj < 8; ++jj) acc[jj] = 0.0f;
-        // group order 0, 1, 2: the sum is the same on every run
-        for (int g = 0; g < kDecGroups; ++g) {
-          if (group_first(g, a) > b) continue;     // no step of group g in this segment
+        // groups in order: the sum is the same on every run
+        for (int g = 0; g < S::kGroups; ++g) {
+          if (group_first(g, a, S::kGroups) > b) continue;   // no step of group g in this segment
           uint32_t v[8];
-          tmem_ld_32x32b_x8(tmem + lane_base + S::kDCol + (set * kDecGroups + g) * NCOL + c0, v);
+          tmem_ld_32x32b_x8(tmem + lane_base + S::kDCol + (set * S::kGroups + g) * NCOL + c0, v);
           tmem_wait_ld();
 #pragma unroll
           for (int jj = 0; jj < 8; ++jj) acc[jj] += __uint_as_float(v[jj]);
