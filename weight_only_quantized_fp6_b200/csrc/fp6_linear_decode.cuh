@@ -74,8 +74,13 @@ struct DecodeShape {
   static constexpr int kSlotCols = kTMax * 32;
   static constexpr int kDCol = kSlots * kSlotCols;          // accumulators after the slots
   // accumulator sets: two (segments alternate) when they fit in TMEM
-  static constexpr int kSets = (kDCol + 2 * kGroups * NCOL <= static_cast<int>(kTmemCols)) ? 2 : 1;
-  static constexpr int kAccCols = kSets * kGroups * NCOL;   // [set][group][NCOL]
+  // MMA-issuing warps per group: each issues the k-slices 4/kIss*i .. of every
+  // tile of the step into its own accumulator.  One thread issues one MMA in
+  // about 160 cycles, so two issuers halve the group's issue time where TMEM
+  // has room for their accumulators (16 token columns).
+  static constexpr int kIss = (NCOL == 16) ? 2 : 1;
+  static constexpr int kSets = (kDCol + 2 * kGroups * kIss * NCOL <= static_cast<int>(kTmemCols)) ? 2 : 1;
+  static constexpr int kAccCols = kSets * kGroups * kIss * NCOL;   // [set][group][issuer][NCOL]
   static constexpr int kWOff = kRX * kXStage;
   static constexpr int kBarOff = kWOff + kSW * kWStage;
   // wfull, wempty [SW]; xfull, xempty [RX]; slot free [6]; dfull, dempty [2]; epi [2]; done
@@ -146,11 +151,12 @@ __global__ void __launch_bounds__(DecodeShape<NCOL>::kThreads, 1)
   if (threadIdx.x < S::kNumBars) {
     const int b = threadIdx.x;
     const int bx = 2 * kSW, bs = bx + 2 * kRX, bd = bs + S::kSlots;
-    uint32_t count = 1;                                       // wfull, xfull, xempty, slotfree
+    uint32_t count = 1;                                       // wfull, xfull
     if (b >= kSW && b < bx) count = 4;                        // wempty: the group's four warps
-    else if (b >= bd && b < bd + 2) count = S::kGroups;       // dfull: one arrival per group
+    else if (b >= bx + kRX && b < bd) count = S::kIss;        // xempty, slotfree: the group's issuers
+    else if (b >= bd && b < bd + 2) count = S::kGroups * S::kIss;  // dfull: one arrival per issuer
     else if (b >= bd + 2 && b < bd + 6) count = 4;            // dempty, epi: epilogue warps
-    else if (b == bd + 6) count = S::kGroups;                 // done: one commit per group
+    else if (b == bd + 6) count = S::kGroups * S::kIss;       // done: one commit per issuer
     mbar_init(smem_u32(&bars[b]), count);
     fence_barrier_init();
   }
@@ -218,7 +224,12 @@ __global__ void __launch_bounds__(DecodeShape<NCOL>::kThreads, 1)
     const int g = warp >> 2;
     const int quad = warp & 3;               // TMEM lanes 32*quad .. 32*quad+31
     const int r = quad * 32 + lane;          // weight row within the tile
-    const bool issuer = (quad == g);
+    // issuer index of this warp in its group (-1: not an issuer); the issuers
+    // of the three groups sit on different SM sub-partitions
+    const int iss = (quad == g) ? 0 : (S::kIss == 2 && quad == ((g + 2) & 3)) ? 1 : -1;
+    const bool issuer = iss >= 0;
+    constexpr int kSlice = 4 / S::kIss;      // k-slices of a tile per issuer
+    const int kk0 = (iss < 0 ? 0 : iss) * kSlice;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     constexpr uint32_t idesc = idesc_f16_f32(128, NCOL);
     bool ok = true;
@@ -227,7 +238,7 @@ __global__ void __launch_bounds__(DecodeShape<NCOL>::kThreads, 1)
       int a, b;
       segment_range(sg, tile_first, s0, KS, n_local, &a, &b);
       const int set = sg % S::kSets;
-      const uint32_t d_tmem = tmem + S::kDCol + (set * S::kGroups + g) * NCOL;
+      const uint32_t d_tmem = tmem + S::kDCol + ((set * S::kGroups + g) * S::kIss + (iss < 0 ? 0 : iss)) * NCOL;
       // The accumulators of this set were last used kSets segments ago: the
       // epilogue must have read them before the first MMA or arrival.
       if (issuer && sg >= S::kSets)
@@ -264,9 +275,11 @@ __global__ void __launch_bounds__(DecodeShape<NCOL>::kThreads, 1)
               for (int t = 0; t < T; ++t) {
                 const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(t * (S::kXTile >> 4));
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
+                for (int q = 0; q < kSlice; ++q) {
+                  const int kk = kk0 + q;
                   mma_f16_ts(d_tmem, a0 + t * 32 + kk * 8, bdesc + static_cast<uint64_t>(kk * 2), idesc,
-                             (first && t == 0 && kk == 0) ? 0u : 1u);
+                             (first && t == 0 && q == 0) ? 0u : 1u);
+                }
               }
             }
             tc_commit(smem_u32(&slotfree[slot]));
@@ -348,11 +361,13 @@ __global__ void __launch_bounds__(DecodeShape<NCOL>::kThreads, 1)
         // groups in order: the sum is the same on every run
         for (int g = 0; g < S::kGroups; ++g) {
           if (group_first(g, a, S::kGroups) > b) continue;   // no step of group g in this segment
-          uint32_t v[8];
-          tmem_ld_32x32b_x8(tmem + lane_base + S::kDCol + (set * S::kGroups + g) * NCOL + c0, v);
-          tmem_wait_ld();
+          for (int i = 0; i < S::kIss; ++i) {
+            uint32_t v[8];
+            tmem_ld_32x32b_x8(tmem + lane_base + S::kDCol + ((set * S::kGroups + g) * S::kIss + i) * NCOL + c0, v);
+            tmem_wait_ld();
 #pragma unroll
-          for (int jj = 0; jj < 8; ++jj) acc[jj] += __uint_as_float(v[jj]);
+            for (int jj = 0; jj < 8; ++jj) acc[jj] += __uint_as_float(v[jj]);
+          }
         }
         if (split && !finisher) {
 #pragma unroll
