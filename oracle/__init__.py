@@ -63,6 +63,20 @@ def _load():
             for f in ("oracle_quantize", "oracle_prepack", "oracle_unpack",
                       "oracle_dequant", "oracle_linear"):
                 getattr(lib, f).restype = ctypes.c_int
+            I = ctypes.c_int
+            lib.oracle_fpx_codes.argtypes = [I]
+            lib.oracle_fpx_decode_table.argtypes = [I, P]
+            lib.oracle_fpx_round.argtypes = [I, ctypes.c_double]
+            lib.oracle_fpx_quantize.argtypes = [I, P, I64, I64, P, P]
+            lib.oracle_fpx_packed_bytes.argtypes = [I, I64, I64]
+            lib.oracle_fpx_packed_bytes.restype = I64
+            lib.oracle_fpx_prepack.argtypes = [I, P, I64, I64, P]
+            lib.oracle_fpx_unpack.argtypes = [I, P, I64, I64, P]
+            lib.oracle_fpx_dequant.argtypes = [I, P, P, I64, I64, P]
+            lib.oracle_fpx_linear.argtypes = [I, P, P, P, I64, I64, I64, P]
+            for f in ("oracle_fpx_codes", "oracle_fpx_decode_table", "oracle_fpx_round", "oracle_fpx_quantize",
+                      "oracle_fpx_prepack", "oracle_fpx_unpack", "oracle_fpx_dequant", "oracle_fpx_linear"):
+                getattr(lib, f).restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -159,4 +173,86 @@ def linear(x16: np.ndarray, codes: np.ndarray, scales: np.ndarray, nthreads: int
     st = _load().oracle_linear(_ptr(x16), _ptr(codes), _ptr(scales), M, N, K, _ptr(y), int(nthreads))
     if st != OK:
         raise OracleError(st, "linear")
+    return y
+
+
+# ---- other FPx formats (0 = FP6 e3m2, 1 = FP6 e2m3, 2 = FP4 e2m1) ----------------
+
+E3M2, E2M3, E2M1 = 0, 1, 2
+
+
+def fpx_codes(fmt: int) -> int:
+    return int(_load().oracle_fpx_codes(int(fmt)))
+
+
+def fpx_decode_table(fmt: int) -> np.ndarray:
+    out = np.zeros(fpx_codes(fmt), dtype=np.float64)
+    st = _load().oracle_fpx_decode_table(int(fmt), _ptr(out))
+    if st != OK:
+        raise OracleError(st, "fpx_decode_table")
+    return out
+
+
+def fpx_round(fmt: int, v: float) -> int:
+    return int(_load().oracle_fpx_round(int(fmt), float(v)))
+
+
+def fpx_quantize(fmt: int, W: np.ndarray):
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    N, K = W.shape
+    codes = np.zeros((N, K), dtype=np.uint8)
+    scales = np.zeros(N, dtype=np.uint16)
+    st = _load().oracle_fpx_quantize(int(fmt), _ptr(W), N, K, _ptr(codes), _ptr(scales))
+    if st != OK:
+        raise OracleError(st, "fpx_quantize")
+    return codes, scales
+
+
+def fpx_packed_bytes(fmt: int, N: int, K: int) -> int:
+    return int(_load().oracle_fpx_packed_bytes(int(fmt), N, K))
+
+
+def fpx_prepack(fmt: int, codes: np.ndarray) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    N, K = codes.shape
+    out = np.zeros(fpx_packed_bytes(fmt, N, K), dtype=np.uint8)
+    st = _load().oracle_fpx_prepack(int(fmt), _ptr(codes), N, K, _ptr(out))
+    if st != OK:
+        raise OracleError(st, "fpx_prepack")
+    return out
+
+
+def fpx_unpack(fmt: int, packed: np.ndarray, N: int, K: int) -> np.ndarray:
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    codes = np.zeros((N, K), dtype=np.uint8)
+    st = _load().oracle_fpx_unpack(int(fmt), _ptr(packed), N, K, _ptr(codes))
+    if st != OK:
+        raise OracleError(st, "fpx_unpack")
+    return codes
+
+
+def fpx_dequant(fmt: int, packed: np.ndarray, scales, N: int, K: int) -> np.ndarray:
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    out = np.zeros((N, K), dtype=np.uint16)
+    sp = None
+    if scales is not None:
+        scales = np.ascontiguousarray(scales, dtype=np.uint16)
+        sp = _ptr(scales)
+    st = _load().oracle_fpx_dequant(int(fmt), _ptr(packed), sp, N, K, _ptr(out))
+    if st != OK:
+        raise OracleError(st, "fpx_dequant")
+    return out
+
+
+def fpx_linear(fmt: int, x16: np.ndarray, codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    x16 = np.ascontiguousarray(x16, dtype=np.uint16)
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint16)
+    M, K = x16.shape
+    N, K2 = codes.shape
+    assert K == K2 and scales.shape == (N,)
+    y = np.zeros((M, N), dtype=np.uint16)
+    st = _load().oracle_fpx_linear(int(fmt), _ptr(x16), _ptr(codes), _ptr(scales), M, N, K, _ptr(y))
+    if st != OK:
+        raise OracleError(st, "fpx_linear")
     return y

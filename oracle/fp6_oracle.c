@@ -30,6 +30,11 @@
  *   dequant             pinned: closed form of decode*scale rounded by numpy
  *   linear              pinned: exact rational dot products (tiny shapes),
  *                       one-hot and constant-code special cases
+ *   fpx_* (FP6 e2m3, FP4 e2m1)
+ *                       pinned: closed-form tables over every code, brute-force
+ *                       rounding in exact rationals and CUDA's own host
+ *                       conversions, round trips, an independent reader of the
+ *                       FP4 layout, one-hot probe, exact rational dot products
  */
 #include <math.h>
 #include <stdint.h>
@@ -352,5 +357,222 @@ int oracle_linear(const uint16_t *x, const uint8_t *codes, const uint16_t *scale
     for (int t = 1; t < nthreads; ++t) pthread_create(&th[t], NULL, linear_rows, &jobs[t]);
     linear_rows(&jobs[0]);
     for (int t = 1; t < nthreads; ++t) pthread_join(th[t], NULL);
+    return ORC_OK;
+}
+
+/* ======================================================================== */
+/* Other FPx formats (the pages: one design for floats of several widths)    */
+/* ======================================================================== */
+/*
+ * The FP6-LLM abstract and the TC-FPx article present the kernel design as
+ * covering float weights of several bit widths ("FPx"), and name none of
+ * their bit formats.  Two more formats are taken here, each with one fp16
+ * scale per output row like e3m2 (same readings as for e3m2):
+ *   fmt 1, FP6 e2m3: s = bit 5, e = bits 4..3 (bias 1), m = bits 2..0;
+ *                    e > 0: (-1)^s 2^(e-1) (1 + m/8), e = 0: (-1)^s m/8;
+ *                    largest magnitude 7.5.
+ *   fmt 2, FP4 e2m1: s = bit 3, e = bits 2..1 (bias 1), m = bit 0;
+ *                    e > 0: (-1)^s 2^(e-1) (1 + m/2), e = 0: (-1)^s m/2;
+ *                    largest magnitude 6.
+ * fmt 0 is e3m2 (the functions above).  No format has inf or NaN codes.
+ */
+
+typedef struct { int ebits, mbits, bias; double maxmag; float maxf; } fpx_fmt;
+
+static int fpx_get(int fmt, fpx_fmt *f)
+{
+    switch (fmt) {
+        case 0: *f = (fpx_fmt){3, 2, 3, 28.0, 28.0f}; return 1;
+        case 1: *f = (fpx_fmt){2, 3, 1, 7.5, 7.5f}; return 1;
+        case 2: *f = (fpx_fmt){2, 1, 1, 6.0, 6.0f}; return 1;
+        default: return 0;
+    }
+}
+
+/* Number of codes of the format (2^(1 + e + m)), 0 for an unknown format. */
+int oracle_fpx_codes(int fmt)
+{
+    fpx_fmt f;
+    if (!fpx_get(fmt, &f)) return 0;
+    return 1 << (1 + f.ebits + f.mbits);
+}
+
+/* Value of code c, from the format's definition. */
+static double fpx_decode_one(const fpx_fmt *f, int c)
+{
+    int mb = f->mbits, eb = f->ebits;
+    int s = (c >> (eb + mb)) & 1;
+    int e = (c >> mb) & ((1 << eb) - 1);
+    int m = c & ((1 << mb) - 1);
+    double frac = (double)m / (double)(1 << mb);
+    double mag = (e > 0) ? ldexp(1.0 + frac, e - f->bias) : ldexp(frac, 1 - f->bias);
+    return s ? -mag : mag;
+}
+
+int oracle_fpx_decode_table(int fmt, double *out)
+{
+    fpx_fmt f;
+    if (!fpx_get(fmt, &f)) return ORC_ERR_INVALID_ARG;
+    int n = oracle_fpx_codes(fmt);
+    for (int c = 0; c < n; ++c) out[c] = fpx_decode_one(&f, c);
+    return ORC_OK;
+}
+
+/* Round v to the nearest value of the format, ties to the even mantissa,
+ * saturating at the largest magnitude; the sign of v is kept.  The same steps
+ * as oracle_round_e3m2: subnormal range in units of its spacing, otherwise
+ * the binade of |v| in units of that binade's spacing, round to an integer
+ * with ties to even, rebuild the code (a mantissa carry lands on the next
+ * binade's first code). */
+int oracle_fpx_round(int fmt, double v)
+{
+    fpx_fmt f;
+    if (!fpx_get(fmt, &f)) return -1;
+    int mb = f.mbits, eb = f.ebits;
+    int sign = signbit(v) ? (1 << (eb + mb)) : 0;
+    int maxcode = (1 << (eb + mb)) - 1;
+    double a = fabs(v);
+    int code;
+    if (a < ldexp(1.0, 1 - f.bias)) {
+        code = (int)nearbyint(ldexp(a, f.bias - 1 + mb));   /* subnormal spacing 2^(1-bias-m) */
+    } else {
+        int ex;
+        frexp(a, &ex);
+        int e = ex - 1;                                      /* a in [2^e, 2^(e+1)) */
+        int emax = (1 << eb) - 1 - f.bias;
+        if (e > emax) {
+            code = maxcode + 1;
+        } else {
+            double q = nearbyint(ldexp(a, mb - e));          /* in [2^m, 2^(m+1)] */
+            code = ((e + f.bias) << mb) + ((int)q - (1 << mb));
+        }
+    }
+    if (code > maxcode) code = maxcode;
+    return sign | code;
+}
+
+/* Per row: s = fp16_rne(fp32(amax / maxmag)), code = round(w / s). */
+int oracle_fpx_quantize(int fmt, const float *W, int64_t N, int64_t K, uint8_t *codes, uint16_t *scales)
+{
+    fpx_fmt f;
+    if (!fpx_get(fmt, &f)) return ORC_ERR_INVALID_ARG;
+    if (N < 0 || K < 0) return ORC_ERR_INVALID_ARG;
+    for (int64_t n = 0; n < N; ++n) {
+        const float *row = W + n * K;
+        float amax = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            if (!isfinite(row[k])) return ORC_ERR_NONFINITE;
+            float a = fabsf(row[k]);
+            if (a > amax) amax = a;
+        }
+        if (amax == 0.0f) {
+            scales[n] = 0;
+            memset(codes + n * K, 0, (size_t)K);
+            continue;
+        }
+        volatile float s32 = amax / f.maxf;                  /* IEEE fp32 division */
+        uint16_t s16 = oracle_f64_to_f16_rne((double)s32);
+        if ((s16 & 0x7FFFu) >= 0x7C00u || (s16 & 0x7FFFu) == 0) return ORC_ERR_SCALE_RANGE;
+        scales[n] = s16;
+        double s = oracle_f16_to_f64(s16);
+        for (int64_t k = 0; k < K; ++k) codes[n * K + k] = (uint8_t)oracle_fpx_round(fmt, (double)row[k] / s);
+    }
+    return ORC_OK;
+}
+
+/* Packed size in bytes: 3/4 byte per weight for the 6-bit formats, 1/2 for FP4. */
+int64_t oracle_fpx_packed_bytes(int fmt, int64_t N, int64_t K)
+{
+    if (fmt == 0 || fmt == 1) return N * K / 4 * 3;
+    if (fmt == 2) return N * K / 2;
+    return -1;
+}
+
+/* FP4 packed layout: tiles of 128 rows x 64 columns, 4096 bytes each, stored
+ * like the 6-bit tiles (column-tile index fastest).  Row r of a tile owns
+ * eight 32-bit words F_w at byte (w/4)*2048 + r*16 + (w%4)*4; column kk is in
+ * word kk/8, byte (kk%8)/2, low nibble for even kk and high nibble for odd kk
+ * (each byte holds the pair of codes one conversion instruction turns into an
+ * fp16 pair).  The 6-bit formats use the 6-bit layout above. */
+static inline int64_t fp4_nibble_byte(int64_t n, int64_t k, int64_t K, int *shift)
+{
+    int64_t base = ((n / 128) * (K / 64) + (k / 64)) * 4096;
+    int r = (int)(n % 128), kk = (int)(k % 64), w = kk / 8;
+    *shift = 4 * (kk % 2);
+    return base + (w / 4) * 2048 + r * 16 + (w % 4) * 4 + (kk % 8) / 2;
+}
+
+int oracle_fpx_prepack(int fmt, const uint8_t *codes, int64_t N, int64_t K, uint8_t *packed)
+{
+    if (fmt == 0 || fmt == 1) return oracle_prepack(codes, N, K, packed);
+    if (fmt != 2) return ORC_ERR_INVALID_ARG;
+    if (N < 0 || K < 0) return ORC_ERR_INVALID_ARG;
+    if (N % 128 || K % 64) return ORC_ERR_UNSUPPORTED_SHAPE;
+    memset(packed, 0, (size_t)(N * K / 2));
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) {
+            int sh;
+            int64_t b = fp4_nibble_byte(n, k, K, &sh);
+            packed[b] |= (uint8_t)((codes[n * K + k] & 0xF) << sh);
+        }
+    return ORC_OK;
+}
+
+int oracle_fpx_unpack(int fmt, const uint8_t *packed, int64_t N, int64_t K, uint8_t *codes)
+{
+    if (fmt == 0 || fmt == 1) return oracle_unpack(packed, N, K, codes);
+    if (fmt != 2) return ORC_ERR_INVALID_ARG;
+    if (N < 0 || K < 0) return ORC_ERR_INVALID_ARG;
+    if (N % 128 || K % 64) return ORC_ERR_UNSUPPORTED_SHAPE;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) {
+            int sh;
+            int64_t b = fp4_nibble_byte(n, k, K, &sh);
+            codes[n * K + k] = (uint8_t)((packed[b] >> sh) & 0xF);
+        }
+    return ORC_OK;
+}
+
+int oracle_fpx_dequant(int fmt, const uint8_t *packed, const uint16_t *scales, int64_t N, int64_t K, uint16_t *W16)
+{
+    fpx_fmt f;
+    if (!fpx_get(fmt, &f)) return ORC_ERR_INVALID_ARG;
+    if (N < 0 || K < 0) return ORC_ERR_INVALID_ARG;
+    if (N % 128 || K % 64) return ORC_ERR_UNSUPPORTED_SHAPE;
+    uint8_t *codes = (uint8_t *)malloc((size_t)(N * K) + 1);
+    if (!codes) return ORC_ERR_INVALID_ARG;
+    oracle_fpx_unpack(fmt, packed, N, K, codes);
+    for (int64_t n = 0; n < N; ++n) {
+        double s = scales ? oracle_f16_to_f64(scales[n]) : 1.0;
+        for (int64_t k = 0; k < K; ++k)
+            W16[n * K + k] = oracle_f64_to_f16_rne(fpx_decode_one(&f, codes[n * K + k]) * s);
+    }
+    free(codes);
+    return ORC_OK;
+}
+
+/* The plain definition again, with the format's decode table. */
+int oracle_fpx_linear(int fmt, const uint16_t *x, const uint8_t *codes, const uint16_t *scales,
+                      int64_t M, int64_t N, int64_t K, uint16_t *y)
+{
+    fpx_fmt f;
+    if (!fpx_get(fmt, &f)) return ORC_ERR_INVALID_ARG;
+    if (M < 0 || N < 0 || K < 0) return ORC_ERR_INVALID_ARG;
+    double table[64];
+    oracle_fpx_decode_table(fmt, table);
+    int mask = oracle_fpx_codes(fmt) - 1;
+    double *xr = (double *)malloc(sizeof(double) * (size_t)(K > 0 ? K : 1));
+    if (!xr) return ORC_ERR_INVALID_ARG;
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t k = 0; k < K; ++k) xr[k] = oracle_f16_to_f64(x[m * K + k]);
+        for (int64_t n = 0; n < N; ++n) {
+            double s = oracle_f16_to_f64(scales[n]);
+            const uint8_t *c = codes + n * K;
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k) acc += xr[k] * (s * table[c[k] & mask]);
+            y[m * N + n] = oracle_f64_to_f16_rne(acc);
+        }
+    }
+    free(xr);
     return ORC_OK;
 }
