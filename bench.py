@@ -38,13 +38,18 @@ METRIC = "FP6xFP16 linear: weight GB/s (M<=16) & TFLOP/s (M>=256), % of roofline
 UNIT = "GB/s"
 
 
-def wbytes(N, K):
-    return 0.75 * N * K
+# bytes per weight of each packed format
+FORMAT_BYTES = {"e3m2": 0.75, "e2m3": 0.75, "e2m1": 0.5}
+FORMAT_CODE = {"e3m2": None, "e2m3": 1, "e2m1": 2}
 
 
-def algo_bytes(M, N, K):
+def wbytes(N, K, per_weight=0.75):
+    return per_weight * N * K
+
+
+def algo_bytes(M, N, K, per_weight=0.75):
     """Algorithmic bytes of one launch: packed weights + fp16 scales + fp16 activations."""
-    return 0.75 * N * K + 2 * N + 2 * M * K
+    return per_weight * N * K + 2 * N + 2 * M * K
 
 
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "fp6_linear_decode_kernel_llama70b_o_proj_decode.md")
@@ -503,7 +508,7 @@ def run_fp6(args, world, rank, local):
                                           f"(algorithmic {algo_bytes(prof['M'], N_DIM, K_DIM):.0f} B)")
                          if prof else "no ncu capture of this kernel source",
                          "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs)",
-                         "kernel": "fp6_linear_decode_kernel<16>"},
+                         "kernel": "fp6_linear_decode_kernel<16, Fmt::E3M2>"},
             "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": launches,
@@ -527,7 +532,8 @@ def run_sweep(args):
     """Every layer shape and M of the Llama-70B, OPT-30B and prefill configs:
     per-launch time (a CUDA graph of launches rotating over enough packed-weight
     copies that no launch finds its weights in L2), weight GB/s, TFLOP/s and the
-    fraction of the roofline max(2MNK / P_tensor, (0.75NK + 2N + 2MK) / BW_hbm).
+    fraction of the roofline max(2MNK / P_tensor, (bNK + 2N + 2MK) / BW_hbm),
+    b = 0.75 bytes per weight (FP6) or 0.5 (FP4, --fmt e2m1).
     Weights and activations come from torch's seeded CUDA generator: the
     times do not depend on the values (parity is the tests' job)."""
     import torch
@@ -542,14 +548,15 @@ def run_sweep(args):
     gen.manual_seed(6000)
     stream = torch.cuda.Stream(device=dev)
     ws = fp6.Workspace(dev)
+    fmt, bpw = FORMAT_CODE[args.fmt], FORMAT_BYTES[args.fmt]
     rows = []
     for cfg in (2, 3, 4, 5):
         spec = inputs.CONFIGS[cfg]
         for lname, (N, K) in spec["layers"].items():
             W = torch.randn(N, K, device=dev, generator=gen) * 0.02
-            layer = fp6.FP6Linear.from_float(W)
+            layer = fp6.FP6Linear.from_float(W, fmt=fmt)
             del W
-            copies = max(1, min(8, math.ceil(4 * l2 / wbytes(N, K))))
+            copies = max(1, min(8, math.ceil(4 * l2 / wbytes(N, K, bpw))))
             packs = [layer.packed] + [layer.packed.clone() for _ in range(copies - 1)]
             for M in spec["M"]:
                 x = torch.randn(M, K, device=dev, generator=gen).half()
@@ -557,12 +564,12 @@ def run_sweep(args):
                 ws.get(fp6.workspace_bytes(M, N, K))
                 n_launch = max(2 * copies, 8)
                 with torch.cuda.stream(stream):
-                    fp6.linear(x, packs[0], layer.scales, N, K, out=y, workspace=ws)
+                    fp6.linear(x, packs[0], layer.scales, N, K, out=y, workspace=ws, fmt=fmt)
                     stream.synchronize()
                     graph = torch.cuda.CUDAGraph()
                     with torch.cuda.graph(graph, stream=stream):
                         for i in range(n_launch):
-                            fp6.linear(x, packs[i % copies], layer.scales, N, K, out=y, workspace=ws)
+                            fp6.linear(x, packs[i % copies], layer.scales, N, K, out=y, workspace=ws, fmt=fmt)
                     graph.replay()
                     e0 = torch.cuda.Event(enable_timing=True)
                     e1 = torch.cuda.Event(enable_timing=True)
@@ -574,9 +581,9 @@ def run_sweep(args):
                 t = e0.elapsed_time(e1) * 1e-3 / (3 * n_launch)
                 del graph
                 t_tc = 2.0 * M * N * K / (peaks["bf16_tflops"] * 1e12)
-                t_hbm = algo_bytes(M, N, K) / (peaks["hbm_gbs"] * 1e9)
-                rows.append({"config": spec["name"], "layer": lname, "N": N, "K": K, "M": M,
-                             "us": round(t * 1e6, 2), "weight_gbs": round(wbytes(N, K) / t / 1e9, 1),
+                t_hbm = algo_bytes(M, N, K, bpw) / (peaks["hbm_gbs"] * 1e9)
+                rows.append({"config": spec["name"], "format": args.fmt, "layer": lname, "N": N, "K": K, "M": M,
+                             "us": round(t * 1e6, 2), "weight_gbs": round(wbytes(N, K, bpw) / t / 1e9, 1),
                              "tflops": round(2.0 * M * N * K / t / 1e12, 1),
                              "bound": "tensor" if t_tc > t_hbm else "hbm",
                              "roofline_frac": round(max(t_tc, t_hbm) / t, 4)})
@@ -596,6 +603,8 @@ def main():
     ap.add_argument("--impl", choices=["fp6", "reference"], default="fp6")
     ap.add_argument("--sweep", action="store_true",
                     help="time every layer shape and M of the Llama-70B, OPT-30B and prefill configs (1 GPU)")
+    ap.add_argument("--fmt", choices=sorted(FORMAT_BYTES), default="e3m2",
+                    help="weight format of the --sweep (e3m2 = the FP6 layer the bench line times)")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the prefill and two-kernel context measurements (outside the timed region)")
     args = ap.parse_args()

@@ -180,6 +180,43 @@ fp6_status fp6_linear_noalloc(const uint16_t *x, const void *packed, const uint1
  * Returns FP6_OK or an argument error. */
 fp6_status fp6_linear_plan(int64_t M, int64_t N, int64_t K, int64_t out[5]);
 
+/*
+ * Other float formats -- the FP6-LLM pages present the design as one for
+ * float weights of several bit widths (TC-FPx: "x" bits); these entry points
+ * run the same pipeline for two more formats, with the same conventions,
+ * status codes, workspace (fp6_linear_workspace_bytes) and launch rules as
+ * the fp6_* functions.  Each has one FP16 scale per row,
+ *     scale[n] = fp16_rne( fp32( max_k |W[n,k]| / largest ) ),
+ * codes rounded to nearest with ties to even mantissa and saturating.
+ *   FPX_E3M2  the FP6 e3m2 format above (fpx_* with it = the fp6_* calls).
+ *   FPX_E2M3  FP6: sign bit 5, exponent bits 4..3 (bias 1), mantissa bits
+ *             2..0; value (-1)^s 2^(e-1) (1 + m/8), or (-1)^s m/8 for e = 0;
+ *             largest 7.5.  Packed exactly like e3m2 (layout version 2).
+ *   FPX_E2M1  FP4: sign bit 3, exponent bits 2..1 (bias 1), mantissa bit 0;
+ *             value (-1)^s 2^(e-1) (1 + m/2), or (-1)^s m/2 for e = 0;
+ *             largest 6.  Packed N*K/2 bytes: tiles of 128 rows x 64
+ *             columns, tile (nt, kt) at byte (nt*(K/64)+kt)*4096; inside a
+ *             tile row r owns 8 words F_w at byte (w/4)*2048 + r*16 +
+ *             (w%4)*4, and column kk is the 4-bit field at bits
+ *             4*(kk%8) .. 4*(kk%8)+3 of F_{kk/8} (little-endian words: byte
+ *             (kk%8)/2 of the word, low nibble for even kk).
+ * Codes in the [N,K] code buffers are one per byte (unused high bits zero on
+ * output, ignored on input).  An unknown fmt returns FP6_ERR_INVALID_ARG
+ * (fpx_packed_bytes returns 0).
+ */
+typedef enum { FPX_E3M2 = 0, FPX_E2M3 = 1, FPX_E2M1 = 2 } fpx_format;
+
+size_t fpx_packed_bytes(fpx_format fmt, int64_t N, int64_t K);
+fp6_status fpx_quantize(fpx_format fmt, const float *W, int64_t N, int64_t K,
+                        uint8_t *codes, uint16_t *scales, struct CUstream_st *stream);
+fp6_status fpx_prepack(fpx_format fmt, const uint8_t *codes, int64_t N, int64_t K,
+                       void *packed, size_t packed_bytes, struct CUstream_st *stream);
+fp6_status fpx_dequant(fpx_format fmt, const void *packed, const uint16_t *scales, int64_t N, int64_t K,
+                       uint16_t *W16, struct CUstream_st *stream);
+fp6_status fpx_linear(fpx_format fmt, const uint16_t *x, const void *packed, const uint16_t *scales,
+                      int64_t M, int64_t N, int64_t K, uint16_t *y,
+                      void *workspace, size_t workspace_bytes, struct CUstream_st *stream);
+
 #ifdef __cplusplus
 }
 #endif

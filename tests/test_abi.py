@@ -19,7 +19,7 @@ def lib():
 def declared_functions():
     src = open(os.path.join(ROOT, "include", "fp6.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(fp6_[a-z_0-9]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(fp[6x]_[a-z_0-9]+)\s*\(", src)))
 
 
 def test_every_declared_symbol_is_exported(lib):
@@ -72,6 +72,36 @@ def test_host_side_validation(lib):
     assert lib.fp6_linear(None, None, None, 0, 128, 64, ok_ptr, None, 0, None) == 0
     assert lib.fp6_prepack(None, 0, 64, None, 0, None) == 0
     assert lib.fp6_quantize(None, 0, 64, None, None, None) == 0
+
+
+def test_fpx_packed_bytes_and_validation(lib):
+    P = ctypes.c_void_p
+    ok_ptr = P(1 << 20)
+    assert lib.fpx_packed_bytes(0, 8192, 8192) == 50331648      # e3m2
+    assert lib.fpx_packed_bytes(1, 8192, 8192) == 50331648      # e2m3
+    assert lib.fpx_packed_bytes(2, 8192, 8192) == 33554432      # e2m1: half a byte per weight
+    assert lib.fpx_packed_bytes(2, 128, 96) == 0
+    assert lib.fpx_packed_bytes(3, 128, 64) == 0                # unknown format
+    assert lib.fpx_packed_bytes(-1, 128, 64) == 0
+    # unknown format: an argument error before anything else
+    assert lib.fpx_linear(3, ok_ptr, ok_ptr, ok_ptr, 4, 128, 64, ok_ptr, None, 0, None) == 1
+    assert lib.fpx_quantize(7, ok_ptr, 128, 64, ok_ptr, ok_ptr, None) == 1
+    assert lib.fpx_prepack(-1, ok_ptr, 128, 64, ok_ptr, 1 << 20, None) == 1
+    assert lib.fpx_dequant(3, ok_ptr, None, 128, 64, ok_ptr, None) == 1
+    # the shape and buffer rules of the fp6 entry points, per format
+    for fmt in (0, 1, 2):
+        assert lib.fpx_linear(fmt, ok_ptr, ok_ptr, ok_ptr, 4, 100, 64, ok_ptr, None, 0, None) == 2
+        assert lib.fpx_prepack(fmt, ok_ptr, 128, 100, ok_ptr, 1 << 20, None) == 2
+        assert lib.fpx_linear(fmt, ok_ptr, ok_ptr, ok_ptr, 4, 128, 64, P((1 << 20) + 8), None, 0, None) == 3
+        assert lib.fpx_linear(fmt, None, None, None, 0, 128, 64, ok_ptr, None, 0, None) == 0
+    assert lib.fpx_prepack(2, ok_ptr, 128, 64, ok_ptr, 4095, None) == 1   # short buffer (needs 4096)
+    assert lib.fpx_prepack(1, ok_ptr, 128, 64, ok_ptr, 6143, None) == 1
+
+
+def test_python_rejects_unknown_format():
+    import weight_only_quantized_fp6_b200 as fp6
+    with pytest.raises(ValueError):
+        fp6.packed_bytes(128, 64, fmt=5)
 
 
 def test_oracle_is_not_linked_into_the_library():

@@ -7,6 +7,10 @@ the library's CUDA kernels.
     import weight_only_quantized_fp6_b200 as fp6
     layer = fp6.FP6Linear.from_float(W)        # W: [N,K] fp32 on cuda
     y = layer(x)                               # x: [M,K] fp16 on cuda -> [M,N] fp16
+
+Every function takes an optional `fmt`: None (the default) is FP6 e3m2 through
+the fp6_* entry points; E3M2, E2M3 (FP6 with two exponent bits) or E2M1 (FP4)
+select the fpx_* entry points with that format.
 """
 from __future__ import annotations
 
@@ -16,9 +20,18 @@ import threading
 from . import _lib
 
 __all__ = ["quantize", "prepack", "dequant", "linear", "linear_plan", "workspace_bytes",
-           "packed_bytes", "device_status", "FP6Linear", "FP6Error", "Workspace"]
+           "packed_bytes", "device_status", "FP6Linear", "FP6Error", "Workspace",
+           "E3M2", "E2M3", "E2M1"]
 
 FP6Error = _lib.FP6Error
+
+# fpx_format values (include/fp6.h)
+E3M2, E2M3, E2M1 = 0, 1, 2
+
+
+def _check_fmt(fmt):
+    if fmt is not None and fmt not in (E3M2, E2M3, E2M1):
+        raise ValueError(f"unknown format {fmt!r}")
 
 
 def _torch():
@@ -42,45 +55,63 @@ def _need_cuda(name, t, dtype, dim=None):
         raise ValueError(f"{name} must be contiguous")
 
 
-def packed_bytes(N: int, K: int) -> int:
-    return int(_lib.load().fp6_packed_bytes(N, K))
+def packed_bytes(N: int, K: int, fmt=None) -> int:
+    _check_fmt(fmt)
+    if fmt is None:
+        return int(_lib.load().fp6_packed_bytes(N, K))
+    return int(_lib.load().fpx_packed_bytes(fmt, N, K))
 
 
-def quantize(W):
+def quantize(W, fmt=None):
     """W [N,K] fp32 (cuda) -> (codes [N,K] uint8, scales [N] fp16).  Synchronizes."""
     torch = _torch()
+    _check_fmt(fmt)
     _need_cuda("W", W, torch.float32, 2)
     N, K = W.shape
     codes = torch.empty((N, K), dtype=torch.uint8, device=W.device)
     scales = torch.empty((N,), dtype=torch.float16, device=W.device)
-    _lib.check(_lib.load().fp6_quantize(W.data_ptr(), N, K, codes.data_ptr(), scales.data_ptr(),
-                                        _stream(W)), "fp6_quantize")
+    lib = _lib.load()
+    if fmt is None:
+        st = lib.fp6_quantize(W.data_ptr(), N, K, codes.data_ptr(), scales.data_ptr(), _stream(W))
+    else:
+        st = lib.fpx_quantize(fmt, W.data_ptr(), N, K, codes.data_ptr(), scales.data_ptr(), _stream(W))
+    _lib.check(st, "fp6_quantize" if fmt is None else "fpx_quantize")
     return codes, scales
 
 
-def prepack(codes):
-    """codes [N,K] uint8 (cuda) -> packed uint8 buffer of 3*N*K/4 bytes."""
+def prepack(codes, fmt=None):
+    """codes [N,K] uint8 (cuda) -> packed uint8 buffer (3*N*K/4 bytes; N*K/2 for E2M1)."""
     torch = _torch()
     _need_cuda("codes", codes, torch.uint8, 2)
     N, K = codes.shape
-    nbytes = packed_bytes(N, K)
+    nbytes = packed_bytes(N, K, fmt)
     if nbytes == 0 and N * K > 0:
         raise FP6Error(2, "fp6_prepack")
     packed = torch.empty((nbytes,), dtype=torch.uint8, device=codes.device)
-    _lib.check(_lib.load().fp6_prepack(codes.data_ptr(), N, K, packed.data_ptr(), nbytes, _stream(codes)),
-               "fp6_prepack")
+    lib = _lib.load()
+    if fmt is None:
+        st = lib.fp6_prepack(codes.data_ptr(), N, K, packed.data_ptr(), nbytes, _stream(codes))
+    else:
+        st = lib.fpx_prepack(fmt, codes.data_ptr(), N, K, packed.data_ptr(), nbytes, _stream(codes))
+    _lib.check(st, "fp6_prepack" if fmt is None else "fpx_prepack")
     return packed
 
 
-def dequant(packed, scales, N: int, K: int):
-    """packed -> W16 [N,K] fp16; scales None gives the unscaled e3m2 values."""
+def dequant(packed, scales, N: int, K: int, fmt=None):
+    """packed -> W16 [N,K] fp16; scales None gives the unscaled code values."""
     torch = _torch()
+    _check_fmt(fmt)
     _need_cuda("packed", packed, torch.uint8, 1)
     if scales is not None:
         _need_cuda("scales", scales, torch.float16, 1)
     out = torch.empty((N, K), dtype=torch.float16, device=packed.device)
-    _lib.check(_lib.load().fp6_dequant(packed.data_ptr(), scales.data_ptr() if scales is not None else None,
-                                       N, K, out.data_ptr(), _stream(packed)), "fp6_dequant")
+    sp = scales.data_ptr() if scales is not None else None
+    lib = _lib.load()
+    if fmt is None:
+        st = lib.fp6_dequant(packed.data_ptr(), sp, N, K, out.data_ptr(), _stream(packed))
+    else:
+        st = lib.fpx_dequant(fmt, packed.data_ptr(), sp, N, K, out.data_ptr(), _stream(packed))
+    _lib.check(st, "fp6_dequant" if fmt is None else "fpx_dequant")
     return out
 
 
@@ -123,27 +154,32 @@ def _default_workspace(device):
         return _default_ws[key]
 
 
-def linear(x, packed, scales, N: int, K: int, out=None, workspace: Workspace | None = None):
+def linear(x, packed, scales, N: int, K: int, out=None, workspace: Workspace | None = None, fmt=None):
     """y[M,N] = x[M,K] . (scales (.) decode(W))^T in fp16 (fp32 accumulation)."""
     torch = _torch()
+    _check_fmt(fmt)
     _need_cuda("x", x, torch.float16, 2)
     _need_cuda("packed", packed, torch.uint8, 1)
     _need_cuda("scales", scales, torch.float16, 1)
     M, K2 = x.shape
     if K2 != K or scales.shape[0] != N:
         raise ValueError("shape mismatch between x, scales and (N, K)")
-    if N > 0 and K > 0 and packed.numel() < packed_bytes(N, K):
-        raise ValueError(f"packed holds {packed.numel()} bytes; an {N} x {K} weight needs {packed_bytes(N, K)}")
+    if N > 0 and K > 0 and packed.numel() < packed_bytes(N, K, fmt):
+        raise ValueError(f"packed holds {packed.numel()} bytes; an {N} x {K} weight needs "
+                         f"{packed_bytes(N, K, fmt)}")
     if out is None:
         out = torch.empty((M, N), dtype=torch.float16, device=x.device)
     else:
         _need_cuda("out", out, torch.float16, 2)
     need = workspace_bytes(M, N, K)
     ws = (workspace or _default_workspace(x.device)).get(need)
-    _lib.check(_lib.load().fp6_linear(
-        x.data_ptr(), packed.data_ptr(), scales.data_ptr(), M, N, K, out.data_ptr(),
-        ws.data_ptr() if ws is not None else None, ws.numel() if ws is not None else 0, _stream(x)),
-        "fp6_linear")
+    args = (x.data_ptr(), packed.data_ptr(), scales.data_ptr(), M, N, K, out.data_ptr(),
+            ws.data_ptr() if ws is not None else None, ws.numel() if ws is not None else 0, _stream(x))
+    lib = _lib.load()
+    if fmt is None:
+        _lib.check(lib.fp6_linear(*args), "fp6_linear")
+    else:
+        _lib.check(lib.fpx_linear(fmt, *args), "fpx_linear")
     return out
 
 
@@ -155,16 +191,19 @@ def device_status(device=None) -> int:
 
 
 class FP6Linear:
-    """A linear layer whose weight is stored as pre-packed FP6 plus fp16 row scales."""
+    """A linear layer whose weight is stored pre-packed (FP6 e3m2 unless `fmt`
+    says otherwise) plus fp16 row scales."""
 
-    def __init__(self, packed, scales, N: int, K: int):
-        self.packed, self.scales, self.N, self.K = packed, scales, N, K
+    def __init__(self, packed, scales, N: int, K: int, fmt=None):
+        _check_fmt(fmt)
+        self.packed, self.scales, self.N, self.K, self.fmt = packed, scales, N, K, fmt
         self.workspace = Workspace(packed.device)
 
     @classmethod
-    def from_float(cls, W):
-        codes, scales = quantize(W)
-        return cls(prepack(codes), scales, W.shape[0], W.shape[1])
+    def from_float(cls, W, fmt=None):
+        codes, scales = quantize(W, fmt)
+        return cls(prepack(codes, fmt), scales, W.shape[0], W.shape[1], fmt)
 
     def __call__(self, x, out=None):
-        return linear(x, self.packed, self.scales, self.N, self.K, out=out, workspace=self.workspace)
+        return linear(x, self.packed, self.scales, self.N, self.K, out=out, workspace=self.workspace,
+                      fmt=self.fmt)

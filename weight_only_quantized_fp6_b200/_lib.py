@@ -36,6 +36,11 @@ SIGNATURES = {
     "fp6_linear_plan": (_ST, [_I64, _I64, _I64, ctypes.POINTER(_I64)]),
     "fp6_linear_noalloc": (_ST, [_P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "fp6_selftest_wait_timeout": (_ST, [_P]),
+    "fpx_packed_bytes": (_SZ, [_ST, _I64, _I64]),
+    "fpx_quantize": (_ST, [_ST, _P, _I64, _I64, _P, _P, _P]),
+    "fpx_prepack": (_ST, [_ST, _P, _I64, _I64, _P, _SZ, _P]),
+    "fpx_dequant": (_ST, [_ST, _P, _P, _I64, _I64, _P, _P]),
+    "fpx_linear": (_ST, [_ST, _P, _P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
 }
 
 _lock = threading.Lock()

@@ -34,6 +34,7 @@ __global__ void wait_timeout_kernel() {
 namespace {
 
 using fp6::DecodeShape;
+using fp6::Fmt;
 using fp6::LinearShape;
 
 constexpr int kMaxDevices = 64;
@@ -52,7 +53,7 @@ fp6_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FP6_OK : FP6_E
 // ---- per-device cached properties ------------------------------------------
 struct DeviceInfo {
   int sms = 0;
-  bool attrs_set[8] = {false, false, false, false, false, false, false, false};
+  bool attrs_set[3][8] = {};   // [format][kernel variant]: shared-memory limit raised
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -160,18 +161,18 @@ bool make_plan(int64_t M, int64_t N, int64_t K, int sms, Plan* pl) {
 // Launches one variant with programmatic dependent launch: the kernel may
 // begin while the previous kernel in the stream finishes (see the kernel's
 // grid-dependency rules).
-template <int NCOL>
+template <int NCOL, Fmt F>
 fp6_status launch_linear(const CUtensorMap& map, const fp6::LinearParams& prm, cudaStream_t stream, int dev) {
-  auto kern = fp6::fp6_linear_kernel<NCOL>;
-  const int smem = LinearShape<NCOL>::kSmemBytes;
+  auto kern = fp6::fp6_linear_kernel<NCOL, F>;
+  const int smem = LinearShape<NCOL, F>::kSmemBytes;
   const int threads = fp6::kLinearThreads;
   const int idx = NCOL == 16 ? 0 : NCOL == 32 ? 1 : NCOL == 64 ? 2 : NCOL == 128 ? 3 : 4;
   {
     std::lock_guard<std::mutex> lk(g_mu);
-    if (!g_dev[dev].attrs_set[idx]) {
+    if (!g_dev[dev].attrs_set[static_cast<int>(F)][idx]) {
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return FP6_ERR_CUDA;
-      g_dev[dev].attrs_set[idx] = true;
+      g_dev[dev].attrs_set[static_cast<int>(F)][idx] = true;
     }
   }
   cudaLaunchConfig_t cfg = {};
@@ -189,22 +190,22 @@ fp6_status launch_linear(const CUtensorMap& map, const fp6::LinearParams& prm, c
 }
 
 // The decode kernel (one token tile of at most 64 columns), launched the same way.
-template <int NCOL>
+template <int NCOL, Fmt F>
 fp6_status launch_decode(const CUtensorMap& map, const fp6::LinearParams& prm, cudaStream_t stream, int dev) {
-  auto kern = fp6::fp6_linear_decode_kernel<NCOL>;
-  const int smem = DecodeShape<NCOL>::kSmemBytes;
+  auto kern = fp6::fp6_linear_decode_kernel<NCOL, F>;
+  const int smem = DecodeShape<NCOL, F>::kSmemBytes;
   const int idx = NCOL == 16 ? 5 : NCOL == 32 ? 6 : 7;
   {
     std::lock_guard<std::mutex> lk(g_mu);
-    if (!g_dev[dev].attrs_set[idx]) {
+    if (!g_dev[dev].attrs_set[static_cast<int>(F)][idx]) {
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return FP6_ERR_CUDA;
-      g_dev[dev].attrs_set[idx] = true;
+      g_dev[dev].attrs_set[static_cast<int>(F)][idx] = true;
     }
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned int>(prm.grid));
-  cfg.blockDim = dim3(static_cast<unsigned int>(DecodeShape<NCOL>::kThreads));
+  cfg.blockDim = dim3(static_cast<unsigned int>(DecodeShape<NCOL, F>::kThreads));
   cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -216,31 +217,20 @@ fp6_status launch_decode(const CUtensorMap& map, const fp6::LinearParams& prm, c
   return cuda_status(cudaGetLastError());
 }
 
-}  // namespace
-
-extern "C" {
-
-const char* fp6_status_string(fp6_status s) {
-  switch (s) {
-    case FP6_OK: return "FP6_OK";
-    case FP6_ERR_INVALID_ARG: return "FP6_ERR_INVALID_ARG";
-    case FP6_ERR_UNSUPPORTED_SHAPE: return "FP6_ERR_UNSUPPORTED_SHAPE";
-    case FP6_ERR_MISALIGNED: return "FP6_ERR_MISALIGNED";
-    case FP6_ERR_NONFINITE: return "FP6_ERR_NONFINITE";
-    case FP6_ERR_SCALE_RANGE: return "FP6_ERR_SCALE_RANGE";
-    case FP6_ERR_WORKSPACE: return "FP6_ERR_WORKSPACE";
-    case FP6_ERR_CUDA: return "FP6_ERR_CUDA";
-    case FP6_ERR_TIMEOUT: return "FP6_ERR_TIMEOUT";
-  }
-  return "FP6_ERR_UNKNOWN";
+// Packed bytes of an N x K weight in format f (shape already checked).
+size_t packed_bytes_of(Fmt f, int64_t N, int64_t K) {
+  const size_t nk = static_cast<size_t>(N) * static_cast<size_t>(K);
+  return f == Fmt::E2M1 ? nk / 2 : nk / 4 * 3;
 }
 
-size_t fp6_packed_bytes(int64_t N, int64_t K) {
-  if (check_shape(N, K) != FP6_OK) return 0;
-  return static_cast<size_t>(N) * static_cast<size_t>(K) / 4 * 3;
+bool fmt_of(int fmt, Fmt* out) {
+  if (fmt < 0 || fmt > 2) return false;
+  *out = static_cast<Fmt>(fmt);
+  return true;
 }
 
-fp6_status fp6_quantize(const float* W, int64_t N, int64_t K, uint8_t* codes, uint16_t* scales,
+template <Fmt F>
+fp6_status quantize_impl(const float* W, int64_t N, int64_t K, uint8_t* codes, uint16_t* scales,
                         cudaStream_t stream) {
   if (N < 0 || K < 0) return FP6_ERR_INVALID_ARG;
   if (N == 0) return FP6_OK;
@@ -251,7 +241,7 @@ fp6_status fp6_quantize(const float* W, int64_t N, int64_t K, uint8_t* codes, ui
   cudaError_t e = cudaMemcpyToSymbolAsync(fp6::g_quant_error, &zero, sizeof(zero), 0,
                                           cudaMemcpyHostToDevice, stream);
   if (e != cudaSuccess) return FP6_ERR_CUDA;
-  fp6::quantize_kernel<256><<<static_cast<unsigned int>(N), 256, 0, stream>>>(W, K, codes, scales);
+  fp6::quantize_kernel<256, F><<<static_cast<unsigned int>(N), 256, 0, stream>>>(W, K, codes, scales);
   if (cudaGetLastError() != cudaSuccess) return FP6_ERR_CUDA;
   unsigned int flags = 0;
   e = cudaMemcpyFromSymbolAsync(&flags, fp6::g_quant_error, sizeof(flags), 0, cudaMemcpyDeviceToHost, stream);
@@ -262,22 +252,24 @@ fp6_status fp6_quantize(const float* W, int64_t N, int64_t K, uint8_t* codes, ui
   return FP6_OK;
 }
 
-fp6_status fp6_prepack(const uint8_t* codes, int64_t N, int64_t K, void* packed, size_t packed_bytes,
+template <Fmt F>
+fp6_status prepack_impl(const uint8_t* codes, int64_t N, int64_t K, void* packed, size_t packed_bytes,
                        cudaStream_t stream) {
   fp6_status st = check_shape(N, K);
   if (st != FP6_OK) return st;
   if (N == 0 || K == 0) return FP6_OK;
   if (!codes || !packed) return FP6_ERR_INVALID_ARG;
-  if (packed_bytes < fp6_packed_bytes(N, K)) return FP6_ERR_INVALID_ARG;
+  if (packed_bytes < packed_bytes_of(F, N, K)) return FP6_ERR_INVALID_ARG;
   if (!aligned16(codes) || !aligned16(packed)) return FP6_ERR_MISALIGNED;
   const int64_t work = N * (K / fp6::kTileCols);
   const int64_t blocks = (work + 255) / 256;
-  fp6::prepack_kernel<<<static_cast<unsigned int>(blocks), 256, 0, stream>>>(
+  fp6::prepack_kernel<F><<<static_cast<unsigned int>(blocks), 256, 0, stream>>>(
       codes, N, K, static_cast<uint8_t*>(packed));
   return cuda_status(cudaGetLastError());
 }
 
-fp6_status fp6_dequant(const void* packed, const uint16_t* scales, int64_t N, int64_t K, uint16_t* W16,
+template <Fmt F>
+fp6_status dequant_impl(const void* packed, const uint16_t* scales, int64_t N, int64_t K, uint16_t* W16,
                        cudaStream_t stream) {
   fp6_status st = check_shape(N, K);
   if (st != FP6_OK) return st;
@@ -286,42 +278,13 @@ fp6_status fp6_dequant(const void* packed, const uint16_t* scales, int64_t N, in
   if (!aligned16(packed) || !aligned16(W16) || (scales && !aligned16(scales))) return FP6_ERR_MISALIGNED;
   const int64_t work = N * (K / fp6::kTileCols);
   const int64_t blocks = (work + 255) / 256;
-  fp6::dequant_kernel<<<static_cast<unsigned int>(blocks), 256, 0, stream>>>(
+  fp6::dequant_kernel<F><<<static_cast<unsigned int>(blocks), 256, 0, stream>>>(
       static_cast<const uint8_t*>(packed), scales, N, K, W16);
   return cuda_status(cudaGetLastError());
 }
 
-fp6_status fp6_linear_plan(int64_t M, int64_t N, int64_t K, int64_t out[5]) {
-  if (!out) return FP6_ERR_INVALID_ARG;
-  fp6_status st = check_shape(N, K);
-  if (st != FP6_OK) return st;
-  if (M < 0) return FP6_ERR_INVALID_ARG;
-  if (M > INT32_MAX) return FP6_ERR_UNSUPPORTED_SHAPE;
-  int dev = 0;
-  const int sms = current_device_sms(&dev);
-  if (sms <= 0) return FP6_ERR_CUDA;
-  Plan pl;
-  make_plan(M, N, K, sms, &pl);
-  out[0] = pl.ncol;
-  out[1] = pl.stages;
-  out[2] = pl.grid;
-  out[3] = pl.tiles;
-  out[4] = pl.total;
-  return FP6_OK;
-}
-
-size_t fp6_linear_workspace_bytes(int64_t M, int64_t N, int64_t K) {
-  if (check_shape(N, K) != FP6_OK || M < 0 || M > INT32_MAX) return 0;
-  int dev = 0;
-  const int sms = current_device_sms(&dev);
-  if (sms <= 0) return 0;
-  Plan pl;
-  make_plan(M, N, K, sms, &pl);
-  if (pl.grid == 0) return 0;
-  return pl.counter_bytes + pl.partial_bytes;
-}
-
-fp6_status fp6_linear(const uint16_t* x, const void* packed, const uint16_t* scales, int64_t M, int64_t N,
+template <Fmt F>
+fp6_status linear_impl(const uint16_t* x, const void* packed, const uint16_t* scales, int64_t M, int64_t N,
                       int64_t K, uint16_t* y, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   fp6_status st = check_shape(N, K);
   if (st != FP6_OK) return st;
@@ -380,11 +343,137 @@ fp6_status fp6_linear(const uint16_t* x, const void* packed, const uint16_t* sca
   if (cr != CUDA_SUCCESS) return FP6_ERR_CUDA;
 
   switch (pl.ncol) {
-    case 16: return launch_decode<16>(map, prm, stream, dev);
-    case 32: return launch_decode<32>(map, prm, stream, dev);
-    case 64: return launch_decode<64>(map, prm, stream, dev);
-    case 128: return launch_linear<128>(map, prm, stream, dev);
-    default: return launch_linear<256>(map, prm, stream, dev);
+    case 16: return launch_decode<16, F>(map, prm, stream, dev);
+    case 32: return launch_decode<32, F>(map, prm, stream, dev);
+    case 64: return launch_decode<64, F>(map, prm, stream, dev);
+    case 128: return launch_linear<128, F>(map, prm, stream, dev);
+    default: return launch_linear<256, F>(map, prm, stream, dev);
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fp6_status_string(fp6_status s) {
+  switch (s) {
+    case FP6_OK: return "FP6_OK";
+    case FP6_ERR_INVALID_ARG: return "FP6_ERR_INVALID_ARG";
+    case FP6_ERR_UNSUPPORTED_SHAPE: return "FP6_ERR_UNSUPPORTED_SHAPE";
+    case FP6_ERR_MISALIGNED: return "FP6_ERR_MISALIGNED";
+    case FP6_ERR_NONFINITE: return "FP6_ERR_NONFINITE";
+    case FP6_ERR_SCALE_RANGE: return "FP6_ERR_SCALE_RANGE";
+    case FP6_ERR_WORKSPACE: return "FP6_ERR_WORKSPACE";
+    case FP6_ERR_CUDA: return "FP6_ERR_CUDA";
+    case FP6_ERR_TIMEOUT: return "FP6_ERR_TIMEOUT";
+  }
+  return "FP6_ERR_UNKNOWN";
+}
+
+size_t fp6_packed_bytes(int64_t N, int64_t K) {
+  if (check_shape(N, K) != FP6_OK) return 0;
+  return packed_bytes_of(Fmt::E3M2, N, K);
+}
+
+fp6_status fp6_quantize(const float* W, int64_t N, int64_t K, uint8_t* codes, uint16_t* scales,
+                        cudaStream_t stream) {
+  return quantize_impl<Fmt::E3M2>(W, N, K, codes, scales, stream);
+}
+
+fp6_status fp6_prepack(const uint8_t* codes, int64_t N, int64_t K, void* packed, size_t packed_bytes,
+                       cudaStream_t stream) {
+  return prepack_impl<Fmt::E3M2>(codes, N, K, packed, packed_bytes, stream);
+}
+
+fp6_status fp6_dequant(const void* packed, const uint16_t* scales, int64_t N, int64_t K, uint16_t* W16,
+                       cudaStream_t stream) {
+  return dequant_impl<Fmt::E3M2>(packed, scales, N, K, W16, stream);
+}
+
+fp6_status fp6_linear_plan(int64_t M, int64_t N, int64_t K, int64_t out[5]) {
+  if (!out) return FP6_ERR_INVALID_ARG;
+  fp6_status st = check_shape(N, K);
+  if (st != FP6_OK) return st;
+  if (M < 0) return FP6_ERR_INVALID_ARG;
+  if (M > INT32_MAX) return FP6_ERR_UNSUPPORTED_SHAPE;
+  int dev = 0;
+  const int sms = current_device_sms(&dev);
+  if (sms <= 0) return FP6_ERR_CUDA;
+  Plan pl;
+  make_plan(M, N, K, sms, &pl);
+  out[0] = pl.ncol;
+  out[1] = pl.stages;
+  out[2] = pl.grid;
+  out[3] = pl.tiles;
+  out[4] = pl.total;
+  return FP6_OK;
+}
+
+size_t fp6_linear_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (check_shape(N, K) != FP6_OK || M < 0 || M > INT32_MAX) return 0;
+  int dev = 0;
+  const int sms = current_device_sms(&dev);
+  if (sms <= 0) return 0;
+  Plan pl;
+  make_plan(M, N, K, sms, &pl);
+  if (pl.grid == 0) return 0;
+  return pl.counter_bytes + pl.partial_bytes;
+}
+
+fp6_status fp6_linear(const uint16_t* x, const void* packed, const uint16_t* scales, int64_t M, int64_t N,
+                      int64_t K, uint16_t* y, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  return linear_impl<Fmt::E3M2>(x, packed, scales, M, N, K, y, workspace, workspace_bytes, stream);
+}
+
+// ---- other formats (fpx_format) -----------------------------------------------
+size_t fpx_packed_bytes(fpx_format fmt, int64_t N, int64_t K) {
+  Fmt f;
+  if (!fmt_of(fmt, &f) || check_shape(N, K) != FP6_OK) return 0;
+  return packed_bytes_of(f, N, K);
+}
+
+fp6_status fpx_quantize(fpx_format fmt, const float* W, int64_t N, int64_t K, uint8_t* codes, uint16_t* scales,
+                        cudaStream_t stream) {
+  Fmt f;
+  if (!fmt_of(fmt, &f)) return FP6_ERR_INVALID_ARG;
+  switch (f) {
+    case Fmt::E3M2: return quantize_impl<Fmt::E3M2>(W, N, K, codes, scales, stream);
+    case Fmt::E2M3: return quantize_impl<Fmt::E2M3>(W, N, K, codes, scales, stream);
+    default: return quantize_impl<Fmt::E2M1>(W, N, K, codes, scales, stream);
+  }
+}
+
+fp6_status fpx_prepack(fpx_format fmt, const uint8_t* codes, int64_t N, int64_t K, void* packed,
+                       size_t packed_bytes, cudaStream_t stream) {
+  Fmt f;
+  if (!fmt_of(fmt, &f)) return FP6_ERR_INVALID_ARG;
+  switch (f) {
+    case Fmt::E3M2: return prepack_impl<Fmt::E3M2>(codes, N, K, packed, packed_bytes, stream);
+    case Fmt::E2M3: return prepack_impl<Fmt::E2M3>(codes, N, K, packed, packed_bytes, stream);
+    default: return prepack_impl<Fmt::E2M1>(codes, N, K, packed, packed_bytes, stream);
+  }
+}
+
+fp6_status fpx_dequant(fpx_format fmt, const void* packed, const uint16_t* scales, int64_t N, int64_t K,
+                       uint16_t* W16, cudaStream_t stream) {
+  Fmt f;
+  if (!fmt_of(fmt, &f)) return FP6_ERR_INVALID_ARG;
+  switch (f) {
+    case Fmt::E3M2: return dequant_impl<Fmt::E3M2>(packed, scales, N, K, W16, stream);
+    case Fmt::E2M3: return dequant_impl<Fmt::E2M3>(packed, scales, N, K, W16, stream);
+    default: return dequant_impl<Fmt::E2M1>(packed, scales, N, K, W16, stream);
+  }
+}
+
+fp6_status fpx_linear(fpx_format fmt, const uint16_t* x, const void* packed, const uint16_t* scales, int64_t M,
+                      int64_t N, int64_t K, uint16_t* y, void* workspace, size_t workspace_bytes,
+                      cudaStream_t stream) {
+  Fmt f;
+  if (!fmt_of(fmt, &f)) return FP6_ERR_INVALID_ARG;
+  switch (f) {
+    case Fmt::E3M2: return linear_impl<Fmt::E3M2>(x, packed, scales, M, N, K, y, workspace, workspace_bytes, stream);
+    case Fmt::E2M3: return linear_impl<Fmt::E2M3>(x, packed, scales, M, N, K, y, workspace, workspace_bytes, stream);
+    default: return linear_impl<Fmt::E2M1>(x, packed, scales, M, N, K, y, workspace, workspace_bytes, stream);
   }
 }
 

@@ -13,9 +13,9 @@ constexpr unsigned int kQuantNonfinite = 1u;
 constexpr unsigned int kQuantScaleRange = 2u;
 
 // One CTA per weight row: max |w| (rejecting NaN/inf), the fp16 scale
-// fp16_rne(fp32(max/28)), then one code per weight.  Rows are read with
-// 16-byte loads when K is a multiple of 4 and the row is aligned.
-template <int THREADS>
+// fp16_rne(fp32(max/largest)) (largest = 28 for e3m2), then one code per
+// weight.
+template <int THREADS, Fmt F = Fmt::E3M2>
 __global__ void __launch_bounds__(THREADS) quantize_kernel(const float* __restrict__ W, int64_t K,
                                                            uint8_t* __restrict__ codes,
                                                            uint16_t* __restrict__ scales) {
@@ -51,7 +51,7 @@ __global__ void __launch_bounds__(THREADS) quantize_kernel(const float* __restri
     if (b) {
       atomicOr(&g_quant_error, kQuantNonfinite);
     } else if (m > 0.0f) {
-      const __half h = __float2half_rn(m / 28.0f);
+      const __half h = __float2half_rn(m / Format<F>::kMax);
       sbits = __half_as_ushort(h);
       const uint16_t mag = sbits & 0x7FFFu;
       if (mag >= 0x7C00u || mag == 0) atomicOr(&g_quant_error, kQuantScaleRange);
@@ -64,14 +64,15 @@ __global__ void __launch_bounds__(THREADS) quantize_kernel(const float* __restri
   const float s = s_scale;
   uint8_t* crow = codes + n * K;
   if (s > 0.0f && isfinite(s)) {
-    for (int64_t k = threadIdx.x; k < K; k += THREADS) crow[k] = e3m2_code(row[k], s);
+    for (int64_t k = threadIdx.x; k < K; k += THREADS) crow[k] = quant_code<F>(row[k], s);
   } else {
     for (int64_t k = threadIdx.x; k < K; k += THREADS) crow[k] = 0;
   }
 }
 
 // One thread per (row, 64-column tile): read 64 codes, write the row's 48
-// bytes of the packed tile.
+// bytes (32 for FP4) of the packed tile.
+template <Fmt F = Fmt::E3M2>
 __global__ void __launch_bounds__(256) prepack_kernel(const uint8_t* __restrict__ codes, int64_t N,
                                                       int64_t K, uint8_t* __restrict__ packed) {
   const int64_t KT = K / kTileCols;
@@ -89,18 +90,21 @@ __global__ void __launch_bounds__(256) prepack_kernel(const uint8_t* __restrict_
 #pragma unroll
     for (int b = 0; b < 16; ++b) c[16 * v + b] = static_cast<uint8_t>(w[b >> 2] >> (8 * (b & 3)));
   }
-  uint32_t F[kRowWords];
-  pack_row(c, F);
-  uint8_t* tile = packed + ((n / kTileRows) * KT + kt) * kTileBytes;
+  using Fm = Format<F>;
+  uint32_t Fw[Fm::kRowWords];
+  Fm::pack(c, Fw);
+  uint8_t* tile = packed + ((n / kTileRows) * KT + kt) * Fm::kTileBytes;
   const int r = static_cast<int>(n % kTileRows);
 #pragma unroll
-  for (int u = 0; u < 3; ++u)
-    *reinterpret_cast<uint4*>(tile + u * 2048 + r * 16) = make_uint4(F[4 * u], F[4 * u + 1], F[4 * u + 2], F[4 * u + 3]);
+  for (int u = 0; u < Fm::kRowWords / 4; ++u)
+    *reinterpret_cast<uint4*>(tile + u * 2048 + r * 16) =
+        make_uint4(Fw[4 * u], Fw[4 * u + 1], Fw[4 * u + 2], Fw[4 * u + 3]);
 }
 
 // One thread per (row, tile): splice the row's 64 weights and write them as
 // fp16.  Without scales: decode(c) exactly.  With scales: fp16_rne(decode * s),
-// the product formed exactly in fp32 (at most 3 + 11 significant bits).
+// the product formed exactly in fp32 (at most 4 + 11 significant bits).
+template <Fmt F = Fmt::E3M2>
 __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* __restrict__ packed,
                                                       const uint16_t* __restrict__ scales, int64_t N,
                                                       int64_t K, uint16_t* __restrict__ W16) {
@@ -109,10 +113,11 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* __restrict_
   if (idx >= N * KT) return;
   const int64_t kt = idx / N;
   const int64_t n = idx % N;
-  const uint8_t* tile = packed + ((n / kTileRows) * KT + kt) * kTileBytes;
-  uint32_t F[kRowWords], w[32];
-  load_row_words(tile, static_cast<int>(n % kTileRows), F);
-  splice_row(F, w);
+  using Fm = Format<F>;
+  const uint8_t* tile = packed + ((n / kTileRows) * KT + kt) * Fm::kTileBytes;
+  uint32_t Fw[Fm::kRowWords], w[32];
+  Fm::load(tile, static_cast<int>(n % kTileRows), Fw);
+  Fm::rebuild(Fw, w);
   const float mul = scales ? __half2float(__ushort_as_half(scales[n])) : 1.0f;
   uint16_t* dst = W16 + n * K + kt * kTileCols;
 #pragma unroll

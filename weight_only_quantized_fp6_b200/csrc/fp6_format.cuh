@@ -1,5 +1,6 @@
 // fp6_format.cuh -- FP6 (e3m2) encoding on the device: the packed layout,
-// the register rebuild of fp16 weights, and the quantizer's rounding.
+// the register rebuild of fp16 weights, and the quantizer's rounding; and the
+// same for the other formats (FP6 e2m3, FP4 e2m1) at the end.
 //
 // e3m2 code (low 6 bits of a byte): s = bit 5, e = bits 4..2 (bias 3),
 // m = bits 1..0.  Value (-1)^s 2^(e-3)(1+m/4), or (-1)^s 2^-2 (m/4) for e = 0.
@@ -115,6 +116,133 @@ __device__ __forceinline__ uint8_t e3m2_code(float w, float s) {
     code = up ? c + 1 : code;
   }
   return static_cast<uint8_t>(code | (signbit(w) ? 0x20 : 0));
+}
+
+// ---- formats ------------------------------------------------------------
+// The FP6-LLM pages describe one design for float weights of several widths.
+// Two more formats share this machinery, each with one fp16 scale per row:
+//   FP6 e2m3: s = bit 5, e = bits 4..3 (bias 1), m = bits 2..0, largest 7.5;
+//             the same 6-bit layout, converted by cvt.rn.f16x2.e2m3x2.
+//   FP4 e2m1: s = bit 3, e = bits 2..1 (bias 1), m = bit 0, largest 6;
+//             tiles of 128 rows x 64 columns in 4096 bytes: row r owns words
+//             F_w (w = 0..7) at byte (w/4)*2048 + r*16 + (w%4)*4, and column
+//             kk sits in bits 4(kk%8) .. 4(kk%8)+3 of F_{kk/8} (each byte holds
+//             two codes, low nibble first), converted by cvt.rn.f16x2.e2m1x2.
+enum class Fmt : int { E3M2 = 0, E2M3 = 1, E2M1 = 2 };
+
+// Two e2m3 codes per 16-bit half of w (low six bits of each byte), as
+// cvt_e3m2x4 does for e3m2.
+__device__ __forceinline__ void cvt_e2m3x4(uint32_t w, uint32_t& o0, uint32_t& o1) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "cvt.rn.f16x2.e2m3x2 %0, l;\n\tcvt.rn.f16x2.e2m3x2 %1, h;\n\t}"
+      : "=r"(o0), "=r"(o1)
+      : "r"(w));
+}
+
+// Eight e2m1 codes (two per byte, low nibble first) to four fp16 pairs.
+__device__ __forceinline__ void cvt_e2m1x8(uint32_t w, uint32_t (&o)[4]) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\tcvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\tcvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3])
+      : "r"(w));
+}
+
+template <Fmt F>
+struct Format;
+
+template <>
+struct Format<Fmt::E3M2> {
+  static constexpr int kTileBytes = 6144;
+  static constexpr int kRowWords = 12;
+  static constexpr int kMags = 32;          // magnitudes; the sign bit is kMags
+  static constexpr float kMax = 28.0f;
+  __host__ __device__ static constexpr float magnitude(int c) { return e3m2_magnitude(c); }
+  __device__ static void load(const uint8_t* tile, int r, uint32_t (&F)[kRowWords]) { load_row_words(tile, r, F); }
+  __device__ static void rebuild(const uint32_t (&F)[kRowWords], uint32_t (&out)[32]) { splice_row(F, out); }
+  __device__ static void pack(const uint8_t (&c)[64], uint32_t (&F)[kRowWords]) { pack_row(c, F); }
+};
+
+template <>
+struct Format<Fmt::E2M3> {
+  static constexpr int kTileBytes = 6144;
+  static constexpr int kRowWords = 12;
+  static constexpr int kMags = 32;
+  static constexpr float kMax = 7.5f;
+  __host__ __device__ static constexpr float magnitude(int c) {
+    return (c < 8) ? c * 0.125f : static_cast<float>(1 << ((c >> 3) - 1)) * (1.0f + (c & 7) * 0.125f);
+  }
+  __device__ static void load(const uint8_t* tile, int r, uint32_t (&F)[kRowWords]) { load_row_words(tile, r, F); }
+  __device__ static void rebuild(const uint32_t (&F)[kRowWords], uint32_t (&out)[32]) {
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      const uint32_t f0 = F[3 * g], f1 = F[3 * g + 1], f2 = F[3 * g + 2];
+      const uint32_t u1 = (f2 & 0xC0C0C0C0u) | ((f1 >> 2) & 0x3F3F3F3Fu);
+      const uint32_t u2 = (u1 & 0xF0F0F0F0u) | ((f0 >> 4) & 0x0F0F0F0Fu);
+      const uint32_t t = u2 >> 2;
+      cvt_e2m3x4(f0, out[8 * g + 0], out[8 * g + 1]);
+      cvt_e2m3x4(f1, out[8 * g + 2], out[8 * g + 3]);
+      cvt_e2m3x4(f2, out[8 * g + 4], out[8 * g + 5]);
+      cvt_e2m3x4(t, out[8 * g + 6], out[8 * g + 7]);
+    }
+  }
+  __device__ static void pack(const uint8_t (&c)[64], uint32_t (&F)[kRowWords]) { pack_row(c, F); }
+};
+
+template <>
+struct Format<Fmt::E2M1> {
+  static constexpr int kTileBytes = 4096;
+  static constexpr int kRowWords = 8;
+  static constexpr int kMags = 8;
+  static constexpr float kMax = 6.0f;
+  __host__ __device__ static constexpr float magnitude(int c) {
+    return (c < 2) ? c * 0.5f : static_cast<float>(1 << ((c >> 1) - 1)) * (1.0f + (c & 1) * 0.5f);
+  }
+  __device__ static void load(const uint8_t* tile, int r, uint32_t (&F)[kRowWords]) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const uint4 a = *reinterpret_cast<const uint4*>(tile + u * 2048 + r * 16);
+      F[4 * u + 0] = a.x;
+      F[4 * u + 1] = a.y;
+      F[4 * u + 2] = a.z;
+      F[4 * u + 3] = a.w;
+    }
+  }
+  __device__ static void rebuild(const uint32_t (&F)[kRowWords], uint32_t (&out)[32]) {
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      uint32_t o[4];
+      cvt_e2m1x8(F[w], o);
+#pragma unroll
+      for (int b = 0; b < 4; ++b) out[4 * w + b] = o[b];
+    }
+  }
+  __device__ static void pack(const uint8_t (&c)[64], uint32_t (&F)[kRowWords]) {
+#pragma unroll
+    for (int w = 0; w < kRowWords; ++w) F[w] = 0;
+#pragma unroll
+    for (int kk = 0; kk < 64; ++kk) F[kk >> 3] |= (c[kk] & 0xFu) << (4 * (kk & 7));
+  }
+};
+
+// Code of w for the scale s > 0 in format F: |w|/s rounded to the nearest
+// magnitude, ties to the even code, saturating at the largest; sign copied
+// from w.  Decided with exact comparisons of |w| against midpoint*s (few
+// significant bits, exact in fp32), which is the rounding of the exact
+// quotient |w|/s.
+template <Fmt F>
+__device__ __forceinline__ uint8_t quant_code(float w, float s) {
+  using Fm = Format<F>;
+  const float a = fabsf(w);
+  int code = 0;
+#pragma unroll
+  for (int c = 0; c < Fm::kMags - 1; ++c) {
+    const float mid = 0.5f * (Fm::magnitude(c) + Fm::magnitude(c + 1));
+    const float t = mid * s;
+    const bool up = (a > t) || (a == t && ((c + 1) & 1) == 0);
+    code = up ? c + 1 : code;
+  }
+  return static_cast<uint8_t>(code | (signbit(w) ? Fm::kMags : 0));
 }
 
 }  // namespace fp6

@@ -74,16 +74,19 @@ constexpr int kMaxGrid = 1024;                // persistent CTAs at most (one pe
 constexpr int kCounterBytes = kMaxGrid * 4;
 constexpr uint32_t kTmemCols = 512;
 
-template <int NCOL>
+template <int NCOL, Fmt F = Fmt::E3M2>
 struct LinearShape {
   static_assert(NCOL == 16 || NCOL == 32 || NCOL == 64 || NCOL == 128 || NCOL == 256, "NCOL");
   static constexpr int kTMax = (NCOL <= 32) ? 4 : (NCOL <= 128) ? 2 : 1;   // tiles per step, at most
   static constexpr int kXTile = NCOL * 128;                 // NCOL rows x 64 fp16, 128-byte swizzled
   static constexpr int kXStage = kTMax * kXTile;
+  static constexpr int kTileBytes = Format<F>::kTileBytes;
   static constexpr int kWStage = kTMax * kTileBytes;
   static constexpr int kIssuers = (NCOL <= 32) ? 4 : (NCOL == 64) ? 2 : 1;
   static constexpr int kRX = (NCOL == 16) ? 8 : (NCOL <= 64) ? 4 : 3;     // x stages (>= 3)
-  static constexpr int kSW = (NCOL <= 32) ? 6 : (NCOL == 64) ? 12 : (NCOL == 128) ? 9 : 18;  // weight stages
+  // weight stages of 6-bit tiles; the same bytes in FP4 tiles
+  static constexpr int kSW = ((NCOL <= 32) ? 6 : (NCOL == 64) ? 12 : (NCOL == 128) ? 9 : 18) * 6144 / kTileBytes /
+                             kDeqGroups * kDeqGroups;
   static constexpr int kR = (kTMax == 4) ? 3 : 6;           // TMEM slots
   static constexpr int kSlotCols = kTMax * 32;              // TMEM columns of one slot
   static constexpr int kDCol = kR * kSlotCols;              // accumulators after the slots
@@ -169,10 +172,11 @@ __device__ __forceinline__ void fence_acq_rel_gpu() {
   asm volatile("fence.acq_rel.gpu;" ::: "memory");
 }
 
-template <int NCOL>
+template <int NCOL, Fmt F = Fmt::E3M2>
 __global__ void __launch_bounds__(kLinearThreads, 1)
     fp6_linear_kernel(const __grid_constant__ CUtensorMap tmap_x, const LinearParams p) {
-  using S = LinearShape<NCOL>;
+  using S = LinearShape<NCOL, F>;
+  using Fm = Format<F>;
   constexpr int kR = S::kR;
   constexpr int kRX = S::kRX;
   constexpr int kSW = S::kSW;
@@ -253,7 +257,7 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
     // ---------------- weight producer ----------------
     const uint64_t pol = policy_evict_first();
     StepCursor cur(s0, KS, MT);
-    const uint32_t bytes = static_cast<uint32_t>(T) * kTileBytes;
+    const uint32_t bytes = static_cast<uint32_t>(T) * Fm::kTileBytes;
     int issued = 0;
     for (int li = 0; li < n_local; ++li, cur.next()) {
       const int s = li % kSW;
@@ -262,7 +266,7 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
         const uint32_t fb = smem_u32(&wfull[s]);
         mbar_arrive_expect_tx(fb, bytes);
         bulk_load(smem_u32(smem + S::kWOff + s * S::kWStage),
-                  p.packed + (static_cast<long long>(cur.nt) * KT + static_cast<long long>(cur.ks) * T) * kTileBytes,
+                  p.packed + (static_cast<long long>(cur.nt) * KT + static_cast<long long>(cur.ks) * T) * Fm::kTileBytes,
                   bytes, fb, pol);
       }
       __syncwarp();
@@ -347,9 +351,9 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
       tc_fence_after();
       const uint8_t* wst = smem + S::kWOff + sw * S::kWStage;
       for (int t = 0; t < T; ++t) {
-        uint32_t F[kRowWords], w[32];
-        load_row_words(wst + t * kTileBytes, r, F);
-        splice_row(F, w);
+        uint32_t Fw[Fm::kRowWords], w[32];
+        Fm::load(wst + t * Fm::kTileBytes, r, Fw);
+        Fm::rebuild(Fw, w);
         tmem_st_32x32b_x32(tmem + lane_base + s * S::kSlotCols + t * 32, w);
       }
       __syncwarp();

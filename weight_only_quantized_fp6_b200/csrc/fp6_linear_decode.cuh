@@ -54,7 +54,7 @@
 namespace fp6 {
 
 
-template <int NCOL>
+template <int NCOL, Fmt F = Fmt::E3M2>
 struct DecodeShape {
   static_assert(NCOL == 16 || NCOL == 32 || NCOL == 64, "decode variants: 16, 32 or 64 token columns");
   // dequant groups: three, or two where three groups' TMEM slots and
@@ -67,9 +67,11 @@ struct DecodeShape {
   static constexpr int kTMax = 2;                           // tiles per step, at most
   static constexpr int kXTile = NCOL * 128;                 // NCOL rows x 64 fp16, 128-byte swizzled
   static constexpr int kXStage = kTMax * kXTile;
+  static constexpr int kTileBytes = Format<F>::kTileBytes;
   static constexpr int kWStage = kTMax * kTileBytes;
   static constexpr int kRX = (NCOL == 16) ? 9 : (NCOL == 32) ? 6 : 4;   // x stages
-  static constexpr int kSW = (NCOL == 16) ? 15 : 12;                    // weight stages
+  // weight stages: 15 (12) of 6-bit tiles; the same bytes in FP4 tiles
+  static constexpr int kSW = ((NCOL == 16) ? 15 : 12) * 6144 / kTileBytes / kGroups * kGroups;
   static constexpr int kSlots = 2 * kGroups;               // TMEM slots: two per group
   static constexpr int kSlotCols = kTMax * 32;
   static constexpr int kDCol = kSlots * kSlotCols;          // accumulators after the slots
@@ -108,10 +110,11 @@ __device__ __forceinline__ int group_first(int g, int a, int groups) {
   return a + ((g - a % groups) + groups) % groups;
 }
 
-template <int NCOL>
-__global__ void __launch_bounds__(DecodeShape<NCOL>::kThreads, 1)
+template <int NCOL, Fmt F = Fmt::E3M2>
+__global__ void __launch_bounds__(DecodeShape<NCOL, F>::kThreads, 1)
     fp6_linear_decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const LinearParams p) {
-  using S = DecodeShape<NCOL>;
+  using S = DecodeShape<NCOL, F>;
+  using Fm = Format<F>;
   constexpr int kSW = S::kSW;
   constexpr int kRX = S::kRX;
   extern __shared__ uint8_t smem_raw[];
@@ -181,7 +184,7 @@ __global__ void __launch_bounds__(DecodeShape<NCOL>::kThreads, 1)
     // ---------------- weight producer ----------------
     const uint64_t pol = policy_evict_first();
     StepCursor cur(s0, KS, 1);
-    const uint32_t bytes = static_cast<uint32_t>(T) * kTileBytes;
+    const uint32_t bytes = static_cast<uint32_t>(T) * Fm::kTileBytes;
     int issued = 0;
     for (int li = 0; li < n_local; ++li, cur.next()) {
       const int s = li % kSW;
@@ -190,7 +193,7 @@ __global__ void __launch_bounds__(DecodeShape<NCOL>::kThreads, 1)
         const uint32_t fb = smem_u32(&wfull[s]);
         mbar_arrive_expect_tx(fb, bytes);
         bulk_load(smem_u32(smem + S::kWOff + s * S::kWStage),
-                  p.packed + (static_cast<long long>(cur.nt) * KT + static_cast<long long>(cur.ks) * T) * kTileBytes,
+                  p.packed + (static_cast<long long>(cur.nt) * KT + static_cast<long long>(cur.ks) * T) * Fm::kTileBytes,
                   bytes, fb, pol);
       }
       __syncwarp();
@@ -254,9 +257,9 @@ __global__ void __launch_bounds__(DecodeShape<NCOL>::kThreads, 1)
         if (ok) {
           const uint8_t* wst = smem + S::kWOff + sw * S::kWStage;
           for (int t = 0; t < T; ++t) {
-            uint32_t F[kRowWords], w[32];
-            load_row_words(wst + t * kTileBytes, r, F);
-            splice_row(F, w);
+            uint32_t Fw[Fm::kRowWords], w[32];
+            Fm::load(wst + t * Fm::kTileBytes, r, Fw);
+            Fm::rebuild(Fw, w);
             tmem_st_32x32b_x32(tmem + lane_base + slot * S::kSlotCols + t * 32, w);
           }
         }
