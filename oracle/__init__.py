@@ -176,9 +176,9 @@ def linear(x16: np.ndarray, codes: np.ndarray, scales: np.ndarray, nthreads: int
     return y
 
 
-# ---- other FPx formats (0 = FP6 e3m2, 1 = FP6 e2m3, 2 = FP4 e2m1) ----------------
+# ---- other FPx formats (0 = FP6 e3m2, 1 = FP6 e2m3, 2 = FP4 e2m1, 3 = FP5 e2m2) ----
 
-E3M2, E2M3, E2M1 = 0, 1, 2
+E3M2, E2M3, E2M1, E2M2 = 0, 1, 2, 3
 
 
 def fpx_codes(fmt: int) -> int:

@@ -30,11 +30,13 @@
  *   dequant             pinned: closed form of decode*scale rounded by numpy
  *   linear              pinned: exact rational dot products (tiny shapes),
  *                       one-hot and constant-code special cases
- *   fpx_* (FP6 e2m3, FP4 e2m1)
+ *   fpx_* (FP6 e2m3, FP4 e2m1, FP5 e2m2)
  *                       pinned: closed-form tables over every code, brute-force
  *                       rounding in exact rationals and CUDA's own host
- *                       conversions, round trips, an independent reader of the
- *                       FP4 layout, one-hot probe, exact rational dot products
+ *                       conversions (e2m3, e2m1; e2m2 through its values being
+ *                       e2m3 values), round trips, independent readers of the
+ *                       FP4 and FP5 layouts, one-hot probes, exact rational dot
+ *                       products
  */
 #include <math.h>
 #include <stdint.h>
@@ -374,6 +376,9 @@ int oracle_linear(const uint16_t *x, const uint8_t *codes, const uint16_t *scale
  *   fmt 2, FP4 e2m1: s = bit 3, e = bits 2..1 (bias 1), m = bit 0;
  *                    e > 0: (-1)^s 2^(e-1) (1 + m/2), e = 0: (-1)^s m/2;
  *                    largest magnitude 6.
+ *   fmt 3, FP5 e2m2: s = bit 4, e = bits 3..2 (bias 1), m = bits 1..0;
+ *                    e > 0: (-1)^s 2^(e-1) (1 + m/4), e = 0: (-1)^s m/4;
+ *                    largest magnitude 7.
  * fmt 0 is e3m2 (the functions above).  No format has inf or NaN codes.
  */
 
@@ -385,6 +390,7 @@ static int fpx_get(int fmt, fpx_fmt *f)
         case 0: *f = (fpx_fmt){3, 2, 3, 28.0, 28.0f}; return 1;
         case 1: *f = (fpx_fmt){2, 3, 1, 7.5, 7.5f}; return 1;
         case 2: *f = (fpx_fmt){2, 1, 1, 6.0, 6.0f}; return 1;
+        case 3: *f = (fpx_fmt){2, 2, 1, 7.0, 7.0f}; return 1;
         default: return 0;
     }
 }
@@ -480,12 +486,40 @@ int oracle_fpx_quantize(int fmt, const float *W, int64_t N, int64_t K, uint8_t *
     return ORC_OK;
 }
 
-/* Packed size in bytes: 3/4 byte per weight for the 6-bit formats, 1/2 for FP4. */
+/* Packed size in bytes: 3/4 byte per weight for the 6-bit formats, 1/2 for
+ * FP4, 5/8 for FP5. */
 int64_t oracle_fpx_packed_bytes(int fmt, int64_t N, int64_t K)
 {
     if (fmt == 0 || fmt == 1) return N * K / 4 * 3;
     if (fmt == 2) return N * K / 2;
+    if (fmt == 3) return N * K / 8 * 5;
     return -1;
+}
+
+/* FP5 packed layout (the "4+1" cut of a 5-bit weight: a 4-bit piece and a
+ * 1-bit piece, each kind in its own aligned 32-bit words): tiles of 128 rows x
+ * 64 columns, 5120 bytes each, stored like the other tiles.  Row r of a tile
+ * owns eight words P_w of 4-bit pieces at byte (w/4)*2048 + r*16 + (w%4)*4 and
+ * two words Q_q of 1-bit pieces at byte 4096 + r*8 + q*4.  Column kk is
+ * position i = kk%32 of half q = kk/32; with v = i/8, h = (i%8)/4, b = i%4:
+ *   the code's top four bits (code >> 1) sit at bits 8b+4h .. 8b+4h+3 of
+ *   P_{4q+v}, and its lowest bit (code & 1) at bit 8b+2v+h of Q_q.
+ * (So each byte of a P word holds the pieces of codes b and b+4 of its group of
+ * eight, and the eight bits that complete one P word's codes sit at
+ * positions 8b+2v and 8b+2v+1 of Q.) */
+static inline void fp5_positions(int64_t n, int64_t k, int64_t K, int64_t *pbyte, int *pshift,
+                                 int64_t *qbyte, int *qshift)
+{
+    int64_t base = ((n / 128) * (K / 64) + (k / 64)) * 5120;
+    int r = (int)(n % 128), kk = (int)(k % 64);
+    int q = kk / 32, i = kk % 32, v = i / 8, h = (i % 8) / 4, b = i % 4;
+    int w = 4 * q + v;
+    int pbit = 8 * b + 4 * h;                                /* bit within P_w */
+    int qbit = 8 * b + 2 * v + h;                            /* bit within Q_q */
+    *pbyte = base + (w / 4) * 2048 + r * 16 + (w % 4) * 4 + pbit / 8;
+    *pshift = pbit % 8;
+    *qbyte = base + 4096 + r * 8 + q * 4 + qbit / 8;
+    *qshift = qbit % 8;
 }
 
 /* FP4 packed layout: tiles of 128 rows x 64 columns, 4096 bytes each, stored
@@ -505,9 +539,22 @@ static inline int64_t fp4_nibble_byte(int64_t n, int64_t k, int64_t K, int *shif
 int oracle_fpx_prepack(int fmt, const uint8_t *codes, int64_t N, int64_t K, uint8_t *packed)
 {
     if (fmt == 0 || fmt == 1) return oracle_prepack(codes, N, K, packed);
-    if (fmt != 2) return ORC_ERR_INVALID_ARG;
+    if (fmt != 2 && fmt != 3) return ORC_ERR_INVALID_ARG;
     if (N < 0 || K < 0) return ORC_ERR_INVALID_ARG;
     if (N % 128 || K % 64) return ORC_ERR_UNSUPPORTED_SHAPE;
+    if (fmt == 3) {
+        memset(packed, 0, (size_t)(N * K / 8 * 5));
+        for (int64_t n = 0; n < N; ++n)
+            for (int64_t k = 0; k < K; ++k) {
+                int64_t pb, qb;
+                int ps, qs;
+                fp5_positions(n, k, K, &pb, &ps, &qb, &qs);
+                uint8_t c = codes[n * K + k] & 0x1F;
+                packed[pb] |= (uint8_t)((c >> 1) << ps);
+                packed[qb] |= (uint8_t)((c & 1) << qs);
+            }
+        return ORC_OK;
+    }
     memset(packed, 0, (size_t)(N * K / 2));
     for (int64_t n = 0; n < N; ++n)
         for (int64_t k = 0; k < K; ++k) {
@@ -521,9 +568,19 @@ int oracle_fpx_prepack(int fmt, const uint8_t *codes, int64_t N, int64_t K, uint
 int oracle_fpx_unpack(int fmt, const uint8_t *packed, int64_t N, int64_t K, uint8_t *codes)
 {
     if (fmt == 0 || fmt == 1) return oracle_unpack(packed, N, K, codes);
-    if (fmt != 2) return ORC_ERR_INVALID_ARG;
+    if (fmt != 2 && fmt != 3) return ORC_ERR_INVALID_ARG;
     if (N < 0 || K < 0) return ORC_ERR_INVALID_ARG;
     if (N % 128 || K % 64) return ORC_ERR_UNSUPPORTED_SHAPE;
+    if (fmt == 3) {
+        for (int64_t n = 0; n < N; ++n)
+            for (int64_t k = 0; k < K; ++k) {
+                int64_t pb, qb;
+                int ps, qs;
+                fp5_positions(n, k, K, &pb, &ps, &qb, &qs);
+                codes[n * K + k] = (uint8_t)((((packed[pb] >> ps) & 0xF) << 1) | ((packed[qb] >> qs) & 1));
+            }
+        return ORC_OK;
+    }
     for (int64_t n = 0; n < N; ++n)
         for (int64_t k = 0; k < K; ++k) {
             int sh;

@@ -1,11 +1,12 @@
-"""Pins for the oracle's other FPx formats: FP6 e2m3 (format 1) and FP4 e2m1
-(format 2), each with one fp16 scale per output row.
+"""Pins for the oracle's other FPx formats: FP6 e2m3 (format 1), FP4 e2m1
+(format 2) and FP5 e2m2 (format 3), each with one fp16 scale per output row.
 
 The FP6-LLM abstract and the TC-FPx article present the kernel design as one
 for float weights of several bit widths, without their bit formats.  The two
 formats here follow the usual sign / exponent / mantissa reading:
   e2m3: s = bit 5, e = bits 4..3 (bias 1), m = bits 2..0, largest value 7.5;
-  e2m1: s = bit 3, e = bits 2..1 (bias 1), m = bit 0,     largest value 6.
+  e2m1: s = bit 3, e = bits 2..1 (bias 1), m = bit 0,     largest value 6;
+  e2m2: s = bit 4, e = bits 3..2 (bias 1), m = bits 1..0, largest value 7.
 Every pin below is computed here from that definition, in exact rationals or
 with numpy / CUDA library routines, never with the oracle's own code.
 """
@@ -19,7 +20,9 @@ import numpy as np
 import pytest
 
 FMTS = {1: dict(ebits=2, mbits=3, bias=1, maxv=Fraction(15, 2)),
-        2: dict(ebits=2, mbits=1, bias=1, maxv=Fraction(6))}
+        2: dict(ebits=2, mbits=1, bias=1, maxv=Fraction(6)),
+        3: dict(ebits=2, mbits=2, bias=1, maxv=Fraction(7))}
+ALL = [1, 2, 3]
 
 
 def closed_form(fmt, c):
@@ -50,7 +53,7 @@ def mags(fmt):
     return [closed_form(fmt, c) for c in range(ncodes(fmt) // 2)]
 
 
-@pytest.mark.parametrize("fmt", [1, 2])
+@pytest.mark.parametrize("fmt", ALL)
 def test_decode_table_closed_form(orc, fmt):
     t = orc.fpx_decode_table(fmt)
     assert len(t) == ncodes(fmt)
@@ -96,7 +99,7 @@ def probe_values(fmt):
     return vals + [-v for v in vals]
 
 
-@pytest.mark.parametrize("fmt", [1, 2])
+@pytest.mark.parametrize("fmt", ALL)
 def test_round_vs_brute_force(orc, fmt):
     for v in probe_values(fmt):
         assert orc.fpx_round(fmt, v) == brute_force_code(fmt, v), (fmt, v)
@@ -131,7 +134,7 @@ def test_round_vs_cuda_library(orc, cuda_cvt, fmt):
         assert orc.fpx_round(fmt, v) == cuda_cvt[fmt](v), (fmt, v)
 
 
-@pytest.mark.parametrize("fmt", [1, 2])
+@pytest.mark.parametrize("fmt", ALL)
 def test_quantize_scale_and_codes(orc, fmt):
     from weight_only_quantized_fp6_b200 import inputs
     W = inputs.weights(21 + fmt, 128, 128)
@@ -147,7 +150,7 @@ def test_quantize_scale_and_codes(orc, fmt):
                 codes[n, k] == brute_force_code(fmt, float(np.float64(W[n, k]) / s[n])), (n, k)
 
 
-@pytest.mark.parametrize("fmt", [1, 2])
+@pytest.mark.parametrize("fmt", ALL)
 def test_quantize_round_trip(orc, fmt):
     """Rows built from codes (one at the largest magnitude each) times a
     power-of-two scale come back with the same codes and scale."""
@@ -217,7 +220,7 @@ def test_e2m3_uses_the_six_bit_layout(orc):
     assert np.array_equal(orc.fpx_prepack(1, codes), orc.prepack(codes))
 
 
-@pytest.mark.parametrize("fmt", [1, 2])
+@pytest.mark.parametrize("fmt", ALL)
 def test_dequant_closed_form(orc, fmt):
     rng = np.random.default_rng(8)
     N, K = 128, 128
@@ -231,7 +234,7 @@ def test_dequant_closed_form(orc, fmt):
     assert np.array_equal(orc.fpx_dequant(fmt, packed, None, N, K), ref1)
 
 
-@pytest.mark.parametrize("fmt", [1, 2])
+@pytest.mark.parametrize("fmt", ALL)
 def test_linear_exact_rational(orc, fmt):
     """Tiny shapes: the sum done in exact rationals, rounded once to fp16."""
     rng = np.random.default_rng(9 + fmt)
@@ -253,7 +256,7 @@ def test_linear_exact_rational(orc, fmt):
             assert got == want or abs(float(got) - float(want)) <= abs(float(want)) * 2.0 ** -10, (m, n)
 
 
-@pytest.mark.parametrize("fmt", [1, 2])
+@pytest.mark.parametrize("fmt", ALL)
 def test_linear_one_hot(orc, fmt):
     rng = np.random.default_rng(12)
     N, K = 16, 64
@@ -266,3 +269,73 @@ def test_linear_one_hot(orc, fmt):
     ref = (table[codes].T * scales.view(np.float16).astype(np.float64)[None, :]).astype(np.float16)
     # values compared (an empty sum of signed zeros is +0: the sign of a zero output is not pinned)
     assert np.array_equal(y.view(np.float16), ref)
+
+
+def test_fp5_values_are_e2m3_values_via_cuda(orc, cuda_cvt):
+    """Every e2m2 value is the e2m3 value of the code shifted left by one (the
+    mantissa gains a zero bit): CUDA's own e2m3 conversion of each e2m2 value
+    returns exactly that code."""
+    t = orc.fpx_decode_table(3)
+    for c in range(32):
+        assert Fraction(t[c]) == closed_form(3, c)
+        if closed_form(3, c) != 0:
+            assert cuda_cvt[1](float(t[c])) == ((c & 0x10) << 1) | ((c & 0x0F) << 1), c
+
+
+def read_fp5_codes(packed, N, K):
+    """Independent reader of the FP5 layout, word by word as a GPU thread reads
+    a row: eight 4-bit-piece words P_w at (w/4)*2048 + r*16 + (w%4)*4 and two
+    1-bit-piece words Q_q at 4096 + r*8 + q*4 in each 5120-byte tile.  For
+    word P_{4q+v}: byte b holds the pieces of codes b (low nibble) and b+4
+    (high nibble) of its group of eight; their low bits are Q_q bits
+    8b+2v and 8b+2v+1."""
+    words = packed.view("<u4")
+    out = np.zeros((N, K), dtype=np.uint8)
+    KT = K // 64
+    r = np.arange(128)
+    for nt in range(N // 128):
+        for kt in range(KT):
+            base = (nt * KT + kt) * 1280                     # words per tile
+            for q in range(2):
+                Q = words[base + 1024 + r * 2 + q]
+                for v in range(4):
+                    w = 4 * q + v
+                    P = words[base + (w // 4) * 512 + r * 4 + (w % 4)]
+                    for h in range(2):
+                        for b in range(4):
+                            kk = 32 * q + 8 * v + 4 * h + b
+                            top = (P >> (8 * b + 4 * h)) & 0xF
+                            low = (Q >> (8 * b + 2 * v + h)) & 1
+                            out[nt * 128:(nt + 1) * 128, kt * 64 + kk] = (top << 1) | low
+    return out
+
+
+def test_fp5_prepack_reader_and_round_trip(orc):
+    rng = np.random.default_rng(13)
+    N, K = 256, 192
+    codes = rng.integers(0, 32, size=(N, K)).astype(np.uint8)
+    packed = orc.fpx_prepack(3, codes)
+    assert packed.size == N * K * 5 // 8 == orc.fpx_packed_bytes(3, N, K)
+    assert np.array_equal(read_fp5_codes(packed, N, K), codes)
+    assert np.array_equal(orc.fpx_unpack(3, packed, N, K), codes)
+
+
+def test_fp5_one_hot_probe(orc):
+    """A code with only its low bit set touches one bit of a Q word; a code
+    with only its top four bits set touches one nibble of a P word."""
+    N, K = 128, 128
+    for (n, k) in [(0, 0), (0, 1), (5, 63), (127, 64), (64, 127), (77, 9), (3, 36)]:
+        t = (n // 128) * (K // 64) + k // 64
+        kk = k % 64
+        q, i = kk // 32, kk % 32
+        v, h, b = i // 8, (i % 8) // 4, i % 4
+        r = n % 128
+        for code, want_off, want_val in [
+                (0x01, 4096 + r * 8 + q * 4 + (8 * b + 2 * v + h) // 8, 1 << ((2 * v + h) % 8)),
+                (0x1E, ((4 * q + v) // 4) * 2048 + r * 16 + ((4 * q + v) % 4) * 4 + b, 0xF << (4 * h))]:
+            codes = np.zeros((N, K), dtype=np.uint8)
+            codes[n, k] = code
+            packed = orc.fpx_prepack(3, codes)
+            nz = np.nonzero(packed)[0]
+            assert list(nz) == [t * 5120 + want_off], (n, k, code)
+            assert packed[nz[0]] == want_val, (n, k, code)
