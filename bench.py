@@ -39,8 +39,8 @@ UNIT = "GB/s"
 
 
 # bytes per weight of each packed format
-FORMAT_BYTES = {"e3m2": 0.75, "e2m3": 0.75, "e2m1": 0.5}
-FORMAT_CODE = {"e3m2": None, "e2m3": 1, "e2m1": 2}
+FORMAT_BYTES = {"e3m2": 0.75, "e2m3": 0.75, "e2m1": 0.5, "e2m2": 0.625}
+FORMAT_CODE = {"e3m2": None, "e2m3": 1, "e2m1": 2, "e2m2": 3}
 
 
 def wbytes(N, K, per_weight=0.75):
@@ -533,7 +533,7 @@ def run_sweep(args):
     per-launch time (a CUDA graph of launches rotating over enough packed-weight
     copies that no launch finds its weights in L2), weight GB/s, TFLOP/s and the
     fraction of the roofline max(2MNK / P_tensor, (bNK + 2N + 2MK) / BW_hbm),
-    b = 0.75 bytes per weight (FP6) or 0.5 (FP4, --fmt e2m1).
+    b = 0.75 bytes per weight (FP6), 0.625 (FP5, --fmt e2m2) or 0.5 (FP4, --fmt e2m1).
     Weights and activations come from torch's seeded CUDA generator: the
     times do not depend on the values (parity is the tests' job)."""
     import torch

@@ -200,11 +200,22 @@ fp6_status fp6_linear_plan(int64_t M, int64_t N, int64_t K, int64_t out[5]);
  *             (w%4)*4, and column kk is the 4-bit field at bits
  *             4*(kk%8) .. 4*(kk%8)+3 of F_{kk/8} (little-endian words: byte
  *             (kk%8)/2 of the word, low nibble for even kk).
+ *   FPX_E2M2  FP5: sign bit 4, exponent bits 3..2 (bias 1), mantissa bits
+ *             1..0; value (-1)^s 2^(e-1) (1 + m/4), or (-1)^s m/4 for e = 0;
+ *             largest 7.  Packed 5*N*K/8 bytes, each code cut into a 4-bit
+ *             and a 1-bit piece: tiles of 128 rows x 64 columns, tile
+ *             (nt, kt) at byte (nt*(K/64)+kt)*5120; inside a tile row r owns
+ *             8 words P_w of 4-bit pieces at byte (w/4)*2048 + r*16 + (w%4)*4
+ *             and 2 words Q_q of 1-bit pieces at byte 4096 + r*8 + q*4.
+ *             Column kk is position i = kk%32 of half q = kk/32; with
+ *             v = i/8, h = (i%8)/4, b = i%4, the code's top four bits are
+ *             bits 8b+4h .. 8b+4h+3 of P_{4q+v} and its lowest bit is bit
+ *             8b+2v+h of Q_q.
  * Codes in the [N,K] code buffers are one per byte (unused high bits zero on
  * output, ignored on input).  An unknown fmt returns FP6_ERR_INVALID_ARG
  * (fpx_packed_bytes returns 0).
  */
-typedef enum { FPX_E3M2 = 0, FPX_E2M3 = 1, FPX_E2M1 = 2 } fpx_format;
+typedef enum { FPX_E3M2 = 0, FPX_E2M3 = 1, FPX_E2M1 = 2, FPX_E2M2 = 3 } fpx_format;
 
 size_t fpx_packed_bytes(fpx_format fmt, int64_t N, int64_t K);
 fp6_status fpx_quantize(fpx_format fmt, const float *W, int64_t N, int64_t K,

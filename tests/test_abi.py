@@ -80,22 +80,24 @@ def test_fpx_packed_bytes_and_validation(lib):
     assert lib.fpx_packed_bytes(0, 8192, 8192) == 50331648      # e3m2
     assert lib.fpx_packed_bytes(1, 8192, 8192) == 50331648      # e2m3
     assert lib.fpx_packed_bytes(2, 8192, 8192) == 33554432      # e2m1: half a byte per weight
+    assert lib.fpx_packed_bytes(3, 8192, 8192) == 41943040      # e2m2: five eighths of a byte
     assert lib.fpx_packed_bytes(2, 128, 96) == 0
-    assert lib.fpx_packed_bytes(3, 128, 64) == 0                # unknown format
+    assert lib.fpx_packed_bytes(4, 128, 64) == 0                # unknown format
     assert lib.fpx_packed_bytes(-1, 128, 64) == 0
     # unknown format: an argument error before anything else
-    assert lib.fpx_linear(3, ok_ptr, ok_ptr, ok_ptr, 4, 128, 64, ok_ptr, None, 0, None) == 1
+    assert lib.fpx_linear(4, ok_ptr, ok_ptr, ok_ptr, 4, 128, 64, ok_ptr, None, 0, None) == 1
     assert lib.fpx_quantize(7, ok_ptr, 128, 64, ok_ptr, ok_ptr, None) == 1
     assert lib.fpx_prepack(-1, ok_ptr, 128, 64, ok_ptr, 1 << 20, None) == 1
-    assert lib.fpx_dequant(3, ok_ptr, None, 128, 64, ok_ptr, None) == 1
+    assert lib.fpx_dequant(4, ok_ptr, None, 128, 64, ok_ptr, None) == 1
     # the shape and buffer rules of the fp6 entry points, per format
-    for fmt in (0, 1, 2):
+    for fmt in (0, 1, 2, 3):
         assert lib.fpx_linear(fmt, ok_ptr, ok_ptr, ok_ptr, 4, 100, 64, ok_ptr, None, 0, None) == 2
         assert lib.fpx_prepack(fmt, ok_ptr, 128, 100, ok_ptr, 1 << 20, None) == 2
         assert lib.fpx_linear(fmt, ok_ptr, ok_ptr, ok_ptr, 4, 128, 64, P((1 << 20) + 8), None, 0, None) == 3
         assert lib.fpx_linear(fmt, None, None, None, 0, 128, 64, ok_ptr, None, 0, None) == 0
     assert lib.fpx_prepack(2, ok_ptr, 128, 64, ok_ptr, 4095, None) == 1   # short buffer (needs 4096)
     assert lib.fpx_prepack(1, ok_ptr, 128, 64, ok_ptr, 6143, None) == 1
+    assert lib.fpx_prepack(3, ok_ptr, 128, 64, ok_ptr, 5119, None) == 1
 
 
 def test_python_rejects_unknown_format():

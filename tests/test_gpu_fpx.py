@@ -1,9 +1,9 @@
-"""GPU fpx_* entry points (FP6 e2m3, FP4 e2m1, and e3m2 through the same
-calls) against the oracle.
+"""GPU fpx_* entry points (FP6 e2m3, FP4 e2m1, FP5 e2m2, and e3m2 through
+the same calls) against the oracle.
 
 Quantize, prepack and dequant are compared byte for byte, with every code at
 every position of a tile (which also fixes which nibble of a byte the FP4
-conversion reads first); the linear layer is compared with the tolerance of
+conversion reads first, and the FP5 rebuild's bit gathering); the linear layer is compared with the tolerance of
 the e3m2 tests, over whole small outputs and on sampled rows and tokens of the
 Llama-70B O-projection shape.
 """
@@ -16,8 +16,8 @@ pytestmark = pytest.mark.gpu
 
 torch = pytest.importorskip("torch")
 
-FORMATS = [0, 1, 2]          # e3m2, e2m3, e2m1
-NAMES = {0: "e3m2", 1: "e2m3", 2: "e2m1"}
+FORMATS = [0, 1, 2, 3]       # e3m2, e2m3, e2m1, e2m2
+NAMES = {0: "e3m2", 1: "e2m3", 2: "e2m1", 3: "e2m2"}
 
 
 @pytest.fixture(scope="module")
@@ -136,7 +136,7 @@ def test_linear_grid_shapes(fp6, orc, fmt, N, K):
         run_linear(fp6, orc, fmt, N, K, M, N + K, M)
 
 
-@pytest.mark.parametrize("fmt", [1, 2])
+@pytest.mark.parametrize("fmt", [1, 2, 3])
 def test_one_hot_bit_exact(fp6, orc, fmt):
     """x = identity rows: y[m,n] = fp16_rne(scale[n] * decode(c[n,m])), exactly
     the oracle's dequantized weight."""
@@ -169,7 +169,7 @@ def test_e3m2_through_fpx_is_the_fp6_path(fp6):
         assert torch.equal(fp6.linear(x, p0, s0, N, K), fp6.linear(x, p1, s1, N, K, fmt=0))
 
 
-@pytest.mark.parametrize("fmt", [1, 2])
+@pytest.mark.parametrize("fmt", [1, 2, 3])
 @pytest.mark.parametrize("M", [1, 16, 64, 1024])
 def test_llama70b_o_proj_sampled(fp6, orc, fmt, M):
     """N = K = 8192 in the launch configuration of the benchmark, on sampled

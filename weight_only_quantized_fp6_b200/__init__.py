@@ -9,8 +9,8 @@ the library's CUDA kernels.
     y = layer(x)                               # x: [M,K] fp16 on cuda -> [M,N] fp16
 
 Every function takes an optional `fmt`: None (the default) is FP6 e3m2 through
-the fp6_* entry points; E3M2, E2M3 (FP6 with two exponent bits) or E2M1 (FP4)
-select the fpx_* entry points with that format.
+the fp6_* entry points; E3M2, E2M3 (FP6 with two exponent bits), E2M1 (FP4)
+or E2M2 (FP5) select the fpx_* entry points with that format.
 """
 from __future__ import annotations
 
@@ -21,16 +21,16 @@ from . import _lib
 
 __all__ = ["quantize", "prepack", "dequant", "linear", "linear_plan", "workspace_bytes",
            "packed_bytes", "device_status", "FP6Linear", "FP6Error", "Workspace",
-           "E3M2", "E2M3", "E2M1"]
+           "E3M2", "E2M3", "E2M1", "E2M2"]
 
 FP6Error = _lib.FP6Error
 
 # fpx_format values (include/fp6.h)
-E3M2, E2M3, E2M1 = 0, 1, 2
+E3M2, E2M3, E2M1, E2M2 = 0, 1, 2, 3
 
 
 def _check_fmt(fmt):
-    if fmt is not None and fmt not in (E3M2, E2M3, E2M1):
+    if fmt is not None and fmt not in (E3M2, E2M3, E2M1, E2M2):
         raise ValueError(f"unknown format {fmt!r}")
 
 
@@ -80,7 +80,7 @@ def quantize(W, fmt=None):
 
 
 def prepack(codes, fmt=None):
-    """codes [N,K] uint8 (cuda) -> packed uint8 buffer (3*N*K/4 bytes; N*K/2 for E2M1)."""
+    """codes [N,K] uint8 (cuda) -> packed uint8 buffer (3*N*K/4 bytes; N*K/2 for E2M1, 5*N*K/8 for E2M2)."""
     torch = _torch()
     _need_cuda("codes", codes, torch.uint8, 2)
     N, K = codes.shape

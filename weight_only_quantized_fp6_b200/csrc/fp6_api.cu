@@ -53,7 +53,7 @@ fp6_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FP6_OK : FP6_E
 // ---- per-device cached properties ------------------------------------------
 struct DeviceInfo {
   int sms = 0;
-  bool attrs_set[3][8] = {};   // [format][kernel variant]: shared-memory limit raised
+  bool attrs_set[4][8] = {};   // [format][kernel variant]: shared-memory limit raised
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -220,11 +220,15 @@ fp6_status launch_decode(const CUtensorMap& map, const fp6::LinearParams& prm, c
 // Packed bytes of an N x K weight in format f (shape already checked).
 size_t packed_bytes_of(Fmt f, int64_t N, int64_t K) {
   const size_t nk = static_cast<size_t>(N) * static_cast<size_t>(K);
-  return f == Fmt::E2M1 ? nk / 2 : nk / 4 * 3;
+  switch (f) {
+    case Fmt::E2M1: return nk / 2;
+    case Fmt::E2M2: return nk / 8 * 5;
+    default: return nk / 4 * 3;
+  }
 }
 
 bool fmt_of(int fmt, Fmt* out) {
-  if (fmt < 0 || fmt > 2) return false;
+  if (fmt < 0 || fmt > 3) return false;
   *out = static_cast<Fmt>(fmt);
   return true;
 }
@@ -439,7 +443,8 @@ fp6_status fpx_quantize(fpx_format fmt, const float* W, int64_t N, int64_t K, ui
   switch (f) {
     case Fmt::E3M2: return quantize_impl<Fmt::E3M2>(W, N, K, codes, scales, stream);
     case Fmt::E2M3: return quantize_impl<Fmt::E2M3>(W, N, K, codes, scales, stream);
-    default: return quantize_impl<Fmt::E2M1>(W, N, K, codes, scales, stream);
+    case Fmt::E2M1: return quantize_impl<Fmt::E2M1>(W, N, K, codes, scales, stream);
+    default: return quantize_impl<Fmt::E2M2>(W, N, K, codes, scales, stream);
   }
 }
 
@@ -450,7 +455,8 @@ fp6_status fpx_prepack(fpx_format fmt, const uint8_t* codes, int64_t N, int64_t 
   switch (f) {
     case Fmt::E3M2: return prepack_impl<Fmt::E3M2>(codes, N, K, packed, packed_bytes, stream);
     case Fmt::E2M3: return prepack_impl<Fmt::E2M3>(codes, N, K, packed, packed_bytes, stream);
-    default: return prepack_impl<Fmt::E2M1>(codes, N, K, packed, packed_bytes, stream);
+    case Fmt::E2M1: return prepack_impl<Fmt::E2M1>(codes, N, K, packed, packed_bytes, stream);
+    default: return prepack_impl<Fmt::E2M2>(codes, N, K, packed, packed_bytes, stream);
   }
 }
 
@@ -461,7 +467,8 @@ fp6_status fpx_dequant(fpx_format fmt, const void* packed, const uint16_t* scale
   switch (f) {
     case Fmt::E3M2: return dequant_impl<Fmt::E3M2>(packed, scales, N, K, W16, stream);
     case Fmt::E2M3: return dequant_impl<Fmt::E2M3>(packed, scales, N, K, W16, stream);
-    default: return dequant_impl<Fmt::E2M1>(packed, scales, N, K, W16, stream);
+    case Fmt::E2M1: return dequant_impl<Fmt::E2M1>(packed, scales, N, K, W16, stream);
+    default: return dequant_impl<Fmt::E2M2>(packed, scales, N, K, W16, stream);
   }
 }
 
@@ -473,7 +480,8 @@ fp6_status fpx_linear(fpx_format fmt, const uint16_t* x, const void* packed, con
   switch (f) {
     case Fmt::E3M2: return linear_impl<Fmt::E3M2>(x, packed, scales, M, N, K, y, workspace, workspace_bytes, stream);
     case Fmt::E2M3: return linear_impl<Fmt::E2M3>(x, packed, scales, M, N, K, y, workspace, workspace_bytes, stream);
-    default: return linear_impl<Fmt::E2M1>(x, packed, scales, M, N, K, y, workspace, workspace_bytes, stream);
+    case Fmt::E2M1: return linear_impl<Fmt::E2M1>(x, packed, scales, M, N, K, y, workspace, workspace_bytes, stream);
+    default: return linear_impl<Fmt::E2M2>(x, packed, scales, M, N, K, y, workspace, workspace_bytes, stream);
   }
 }
 

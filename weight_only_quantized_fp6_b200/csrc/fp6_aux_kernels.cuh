@@ -71,7 +71,7 @@ __global__ void __launch_bounds__(THREADS) quantize_kernel(const float* __restri
 }
 
 // One thread per (row, 64-column tile): read 64 codes, write the row's 48
-// bytes (32 for FP4) of the packed tile.
+// bytes (32 for FP4, 40 for FP5) of the packed tile.
 template <Fmt F = Fmt::E3M2>
 __global__ void __launch_bounds__(256) prepack_kernel(const uint8_t* __restrict__ codes, int64_t N,
                                                       int64_t K, uint8_t* __restrict__ packed) {
@@ -94,11 +94,7 @@ __global__ void __launch_bounds__(256) prepack_kernel(const uint8_t* __restrict_
   uint32_t Fw[Fm::kRowWords];
   Fm::pack(c, Fw);
   uint8_t* tile = packed + ((n / kTileRows) * KT + kt) * Fm::kTileBytes;
-  const int r = static_cast<int>(n % kTileRows);
-#pragma unroll
-  for (int u = 0; u < Fm::kRowWords / 4; ++u)
-    *reinterpret_cast<uint4*>(tile + u * 2048 + r * 16) =
-        make_uint4(Fw[4 * u], Fw[4 * u + 1], Fw[4 * u + 2], Fw[4 * u + 3]);
+  Fm::store(tile, static_cast<int>(n % kTileRows), Fw);
 }
 
 // One thread per (row, tile): splice the row's 64 weights and write them as

@@ -128,7 +128,33 @@ __device__ __forceinline__ uint8_t e3m2_code(float w, float s) {
 //             F_w (w = 0..7) at byte (w/4)*2048 + r*16 + (w%4)*4, and column
 //             kk sits in bits 4(kk%8) .. 4(kk%8)+3 of F_{kk/8} (each byte holds
 //             two codes, low nibble first), converted by cvt.rn.f16x2.e2m1x2.
-enum class Fmt : int { E3M2 = 0, E2M3 = 1, E2M1 = 2 };
+//   FP5 e2m2: s = bit 4, e = bits 3..2 (bias 1), m = bits 1..0, largest 7.
+//             Every e2m2 value is the e2m3 value of the code shifted left by
+//             one, so the rebuild forms those e2m3 codes in bytes and converts
+//             them with cvt.rn.f16x2.e2m3x2.  Tiles of 128 rows x 64 columns in
+//             5120 bytes, each code cut 4+1: row r owns eight words P_w of
+//             4-bit pieces (the code's top four bits) at byte
+//             (w/4)*2048 + r*16 + (w%4)*4 and two words Q_q of 1-bit pieces
+//             (its lowest bit) at byte 4096 + r*8 + q*4.  Column kk is
+//             position i = kk%32 of half q = kk/32; with v = i/8, h = (i%8)/4,
+//             b = i%4 its top bits sit at bits 8b+4h.. of P_{4q+v} and its low
+//             bit at bit 8b+2v+h of Q_q.  A P word shifted by two (left for
+//             the low nibbles, right for the high ones) puts four top pieces
+//             in bits 5..2 of four bytes, and Q shifted by 2v-1 (2v) puts
+//             their low bits in bit 1: the e2m3 codes, ready to convert.
+enum class Fmt : int { E3M2 = 0, E2M3 = 1, E2M1 = 2, E2M2 = 3 };
+
+// Store a row's words into a tile laid out as 2048-byte blocks of 16 bytes
+// per row (first 4*(W/4) words), then, for W = 10, one 1024-byte block of
+// 8 bytes per row.
+template <int W>
+__device__ __forceinline__ void store_row_words(uint8_t* tile, int r, const uint32_t (&F)[W]) {
+#pragma unroll
+  for (int u = 0; u < W / 4; ++u)
+    *reinterpret_cast<uint4*>(tile + u * 2048 + r * 16) = make_uint4(F[4 * u], F[4 * u + 1], F[4 * u + 2], F[4 * u + 3]);
+  if constexpr (W % 4 == 2)
+    *reinterpret_cast<uint2*>(tile + (W / 4) * 2048 + r * 8) = make_uint2(F[W - 2], F[W - 1]);
+}
 
 // Two e2m3 codes per 16-bit half of w (low six bits of each byte), as
 // cvt_e3m2x4 does for e3m2.
@@ -161,6 +187,7 @@ struct Format<Fmt::E3M2> {
   __device__ static void load(const uint8_t* tile, int r, uint32_t (&F)[kRowWords]) { load_row_words(tile, r, F); }
   __device__ static void rebuild(const uint32_t (&F)[kRowWords], uint32_t (&out)[32]) { splice_row(F, out); }
   __device__ static void pack(const uint8_t (&c)[64], uint32_t (&F)[kRowWords]) { pack_row(c, F); }
+  __device__ static void store(uint8_t* tile, int r, const uint32_t (&F)[kRowWords]) { store_row_words(tile, r, F); }
 };
 
 template <>
@@ -187,6 +214,7 @@ struct Format<Fmt::E2M3> {
     }
   }
   __device__ static void pack(const uint8_t (&c)[64], uint32_t (&F)[kRowWords]) { pack_row(c, F); }
+  __device__ static void store(uint8_t* tile, int r, const uint32_t (&F)[kRowWords]) { store_row_words(tile, r, F); }
 };
 
 template <>
@@ -223,6 +251,57 @@ struct Format<Fmt::E2M1> {
 #pragma unroll
     for (int kk = 0; kk < 64; ++kk) F[kk >> 3] |= (c[kk] & 0xFu) << (4 * (kk & 7));
   }
+  __device__ static void store(uint8_t* tile, int r, const uint32_t (&F)[kRowWords]) { store_row_words(tile, r, F); }
+};
+
+template <>
+struct Format<Fmt::E2M2> {
+  static constexpr int kTileBytes = 5120;
+  static constexpr int kRowWords = 10;
+  static constexpr int kMags = 16;
+  static constexpr float kMax = 7.0f;
+  __host__ __device__ static constexpr float magnitude(int c) {
+    return (c < 4) ? c * 0.25f : static_cast<float>(1 << ((c >> 2) - 1)) * (1.0f + (c & 3) * 0.25f);
+  }
+  __device__ static void load(const uint8_t* tile, int r, uint32_t (&F)[kRowWords]) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const uint4 a = *reinterpret_cast<const uint4*>(tile + u * 2048 + r * 16);
+      F[4 * u + 0] = a.x;
+      F[4 * u + 1] = a.y;
+      F[4 * u + 2] = a.z;
+      F[4 * u + 3] = a.w;
+    }
+    const uint2 q = *reinterpret_cast<const uint2*>(tile + 4096 + r * 8);
+    F[8] = q.x;
+    F[9] = q.y;
+  }
+  __device__ static void rebuild(const uint32_t (&F)[kRowWords], uint32_t (&out)[32]) {
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const uint32_t Q = F[8 + q];
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const uint32_t P = F[4 * q + v];
+        const uint32_t lo_bits = (v == 0) ? (Q << 1) : (Q >> (2 * v - 1));
+        const uint32_t lo = ((P << 2) & 0x3C3C3C3Cu) | (lo_bits & 0x02020202u);
+        const uint32_t hi = ((P >> 2) & 0x3C3C3C3Cu) | ((Q >> (2 * v)) & 0x02020202u);
+        cvt_e2m3x4(lo, out[16 * q + 4 * v + 0], out[16 * q + 4 * v + 1]);
+        cvt_e2m3x4(hi, out[16 * q + 4 * v + 2], out[16 * q + 4 * v + 3]);
+      }
+    }
+  }
+  __device__ static void pack(const uint8_t (&c)[64], uint32_t (&F)[kRowWords]) {
+#pragma unroll
+    for (int w = 0; w < kRowWords; ++w) F[w] = 0;
+#pragma unroll
+    for (int kk = 0; kk < 64; ++kk) {
+      const int q = kk >> 5, i = kk & 31, v = i >> 3, h = (i >> 2) & 1, b = i & 3;
+      F[4 * q + v] |= ((c[kk] >> 1) & 0xFu) << (8 * b + 4 * h);
+      F[8 + q] |= (c[kk] & 1u) << (8 * b + 2 * v + h);
+    }
+  }
+  __device__ static void store(uint8_t* tile, int r, const uint32_t (&F)[kRowWords]) { store_row_words(tile, r, F); }
 };
 
 // Code of w for the scale s > 0 in format F: |w|/s rounded to the nearest

@@ -1,5 +1,5 @@
 // fp6_linear_decode.cuh -- the FP6 x FP16 linear layer for one token tile of
-// at most 32 tokens (decode), sm_100a.
+// at most 64 tokens (decode), sm_100a.
 //
 // Same product and the same work split as fp6_linear_kernel (fp6_linear.cuh):
 // y[M,N] = x[M,K] . (scale (.) decode(W[N,K]))^T, fp32 accumulation, fp16 out,
@@ -12,19 +12,21 @@
 //   warps 0..4G-1 G dequant groups of four warps (one per TMEM lane
 //                 quadrant), taking every G-th step (G = 3; G = 2 for 64 token
 //                 columns, where three groups' TMEM would not fit).  A group splices its
-//                 step's T tiles into one of its own two TMEM slots, meets on a
-//                 hardware named barrier, and one warp of the group (quadrant
-//                 g, so the three groups issue from three different SM
-//                 sub-partitions) issues the step's 4T MMAs into the group's
-//                 own accumulator.  No hand-off to a separate issuer warp: the
-//                 step's dequant-to-MMA path is one barrier, and the slot it
-//                 refills next was released by the group's own commit two
-//                 steps earlier, long done.
-//   warps 4G..    epilogue warpgroup (four warps): per segment, the G group
-//                 accumulators summed in group order, * scale, fp16
+//                 step's T tiles into one of its own two TMEM slots; each warp
+//                 then reports the slot written on an mbarrier and goes on to
+//                 the next step, so splicing never waits for MMA issue.
+//   warps 4G..    epilogue warpgroup (four warps): per segment, the group
+//                 accumulators summed in a fixed order, * scale, fp16
 //                 store or split-K partial and fix-up.  Accumulators are double
 //                 buffered across segments where TMEM has room (16 token
 //                 columns), single buffered otherwise.
+//   next warps    MMA issuers, kIss per group (two for 16 token columns, else
+//                 one): each waits for its group's slot and the step's
+//                 activations, issues its share of the step's 4T MMAs into its
+//                 own accumulator and commits, which frees the slot and the x
+//                 stage.  One thread issues an MMA in about 50 cycles, and
+//                 several issuing warps overlap, so the issue of one group's
+//                 step overlaps the splicing of the next.
 //   next warp     weight producer: one bulk copy of T packed tiles per step.
 //   last warp     activation producer: one TMA box per step (T column tiles
 //                 of NCOL rows x 64 columns, 128-byte swizzle, rows at or
@@ -36,12 +38,12 @@
 //                 as soon as its own copies land, whatever was issued after.
 //
 // Ring ownership keeps every mbarrier's waits in phase order: weight stages
-// (SW) and x stages (RX) are multiples of G, so each stage is always used
-// by the same group; TMEM slots and accumulators belong to one group.
+// (SW) are a multiple of G and x stages are the TMEM slots, so each stage is
+// always used by the same group; slots and accumulators belong to one group.
 //
-// Named barriers cannot time out, so the group loops never leave early: a
-// warp whose bounded wait gave up (the abort flag is raised) skips its work
-// but still runs every later barrier, and every other wait returns at once.
+// The role loops never leave early: a warp whose bounded wait gave up (the
+// abort flag is raised) skips its work but still makes every later arrival,
+// and every other wait returns at once.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -60,36 +62,40 @@ struct DecodeShape {
   // dequant groups: three, or two where three groups' TMEM slots and
   // accumulators would not fit in the 512 columns (64 token columns)
   static constexpr int kGroups = (NCOL == 64) ? 2 : 3;
+  // MMA-issuing warps per group: each issues the k-slices 4/kIss*i .. of every
+  // tile of the step into its own accumulator.  Two issuers per group where
+  // TMEM has room for their accumulators (16 token columns).
+  static constexpr int kIss = (NCOL == 16) ? 2 : 1;
   static constexpr int kEpiWarp = 4 * kGroups;              // four epilogue warps
-  static constexpr int kWProdWarp = kEpiWarp + 4;
+  static constexpr int kIssWarp = kEpiWarp + 4;             // kGroups * kIss issuer warps
+  static constexpr int kWProdWarp = kIssWarp + kGroups * kIss;
   static constexpr int kXProdWarp = kWProdWarp + 1;
-  static constexpr int kThreads = 32 * (kXProdWarp + 1);   // 576 (three groups) or 448
+  static constexpr int kThreads = 32 * (kXProdWarp + 1);   // 768, 672 or 512
   static constexpr int kTMax = 2;                           // tiles per step, at most
   static constexpr int kXTile = NCOL * 128;                 // NCOL rows x 64 fp16, 128-byte swizzled
   static constexpr int kXStage = kTMax * kXTile;
   static constexpr int kTileBytes = Format<F>::kTileBytes;
   static constexpr int kWStage = kTMax * kTileBytes;
-  static constexpr int kRX = (NCOL == 16) ? 9 : (NCOL == 32) ? 6 : 4;   // x stages
+  // x stages: one per TMEM slot.  Step li uses slot and x stage
+  // 2*(li % G) + ((li / G) & 1); both are free again once the step's MMAs
+  // have completed, which one commit per issuer reports.
+  static constexpr int kRX = 2 * kGroups;
   // weight stages: 15 (12) of 6-bit tiles; the same bytes in FP4 tiles
   static constexpr int kSW = ((NCOL == 16) ? 15 : 12) * 6144 / kTileBytes / kGroups * kGroups;
   static constexpr int kSlots = 2 * kGroups;               // TMEM slots: two per group
   static constexpr int kSlotCols = kTMax * 32;
   static constexpr int kDCol = kSlots * kSlotCols;          // accumulators after the slots
   // accumulator sets: two (segments alternate) when they fit in TMEM
-  // MMA-issuing warps per group: each issues the k-slices 4/kIss*i .. of every
-  // tile of the step into its own accumulator.  One thread issues one MMA in
-  // about 160 cycles, so two issuers halve the group's issue time where TMEM
-  // has room for their accumulators (16 token columns).
-  static constexpr int kIss = (NCOL == 16) ? 2 : 1;
   static constexpr int kSets = (kDCol + 2 * kGroups * kIss * NCOL <= static_cast<int>(kTmemCols)) ? 2 : 1;
   static constexpr int kAccCols = kSets * kGroups * kIss * NCOL;   // [set][group][issuer][NCOL]
   static constexpr int kWOff = kRX * kXStage;
   static constexpr int kBarOff = kWOff + kSW * kWStage;
-  // wfull, wempty [SW]; xfull, xempty [RX]; slot free [6]; dfull, dempty [2]; epi [2]; done
-  static constexpr int kNumBars = 2 * kSW + 2 * kRX + kSlots + 2 + 2 + 2 + 1;
+  // wfull, wempty [SW]; xfull [RX]; slot free [slots] (frees the x stage too);
+  // slot ready [slots]; dfull, dempty [2]; epi [2]; done
+  static constexpr int kNumBars = 2 * kSW + kRX + 2 * kSlots + 2 + 2 + 2 + 1;
   static constexpr int kBarrierBytes = 1024;
   static constexpr int kSmemBytes = kBarOff + kBarrierBytes + 1024;  // + alignment slack
-  static_assert(kSW % kGroups == 0 && kRX % kGroups == 0, "stages owned by one group");
+  static_assert(kSW % kGroups == 0 && kRX == kSlots, "stages owned by one group; one x stage per slot");
   static_assert(kDCol + kAccCols <= static_cast<int>(kTmemCols), "TMEM budget");
   static_assert(kXTile % 1024 == 0 && kTileBytes % 1024 == 0, "1024-byte aligned tiles");
   static_assert(kNumBars * 8 + 32 <= kBarrierBytes, "barrier area");
@@ -123,9 +129,9 @@ __global__ void __launch_bounds__(DecodeShape<NCOL, F>::kThreads, 1)
   uint64_t* wfull = bars;
   uint64_t* wempty = wfull + kSW;
   uint64_t* xfull = wempty + kSW;
-  uint64_t* xempty = xfull + kRX;
-  uint64_t* slotfree = xempty + kRX;              // [6]: a group's MMAs on the slot are done
-  uint64_t* dfull = slotfree + S::kSlots;         // [2]: a segment's accumulators are complete
+  uint64_t* slotfree = xfull + kRX;               // [slots]: a step's MMAs are done (slot and x stage free)
+  uint64_t* slotready = slotfree + S::kSlots;     // [slots]: the group's four warps have written the slot
+  uint64_t* dfull = slotready + S::kSlots;        // [2]: a segment's accumulators are complete
   uint64_t* dempty = dfull + 2;                   // [2]: the epilogue has read them
   uint64_t* epi = dempty + 2;                     // [2]: fix-up meeting (epi[0] only)
   uint64_t* done = epi + 2;                       // every MMA finished (before TMEM release)
@@ -153,10 +159,11 @@ __global__ void __launch_bounds__(DecodeShape<NCOL, F>::kThreads, 1)
 
   if (threadIdx.x < S::kNumBars) {
     const int b = threadIdx.x;
-    const int bx = 2 * kSW, bs = bx + 2 * kRX, bd = bs + S::kSlots;
+    const int bx = 2 * kSW, bs = bx + kRX, br = bs + S::kSlots, bd = br + S::kSlots;
     uint32_t count = 1;                                       // wfull, xfull
     if (b >= kSW && b < bx) count = 4;                        // wempty: the group's four warps
-    else if (b >= bx + kRX && b < bd) count = S::kIss;        // xempty, slotfree: the group's issuers
+    else if (b >= bs && b < br) count = S::kIss;              // slotfree: the group's issuers
+    else if (b >= br && b < bd) count = 4;                    // slotready: the group's four warps
     else if (b >= bd && b < bd + 2) count = S::kGroups * S::kIss;  // dfull: one arrival per issuer
     else if (b >= bd + 2 && b < bd + 6) count = 4;            // dempty, epi: epilogue warps
     else if (b == bd + 6) count = S::kGroups * S::kIss;       // done: one commit per issuer
@@ -209,8 +216,9 @@ __global__ void __launch_bounds__(DecodeShape<NCOL, F>::kThreads, 1)
     int ks = static_cast<int>(s0 - tile_first * KS);
     int issued = 0;
     for (int li = 0; li < n_local; ++li, ks = (ks + 1 == KS) ? 0 : ks + 1) {
-      const int s = li % kRX;
-      if (li >= kRX && !warp_wait(smem_u32(&xempty[s]), ((li / kRX) - 1) & 1, s_abort)) break;
+      const int jg = li / S::kGroups;                         // the step's index in its group
+      const int s = 2 * (li - jg * S::kGroups) + (jg & 1);
+      if (li >= kRX && !warp_wait(smem_u32(&slotfree[s]), ((jg >> 1) - 1) & 1, s_abort)) break;
       if (lane == 0) {
         const uint32_t fb = smem_u32(&xfull[s]);
         mbar_arrive_expect_tx(fb, bytes);
@@ -220,20 +228,57 @@ __global__ void __launch_bounds__(DecodeShape<NCOL, F>::kThreads, 1)
       ++issued;
     }
     // Leave no copy in flight.
-    for (int li = issued > kRX ? issued - kRX : 0; li < issued; ++li)
-      warp_wait(smem_u32(&xfull[li % kRX]), (li / kRX) & 1, s_never);
+    for (int li = issued > kRX ? issued - kRX : 0; li < issued; ++li) {
+      const int jg = li / S::kGroups;
+      warp_wait(smem_u32(&xfull[2 * (li - jg * S::kGroups) + (jg & 1)]), (jg >> 1) & 1, s_never);
+    }
   } else if (warp < 4 * S::kGroups) {
-    // ---------------- dequant groups, each issuing its own MMAs ----------------
+    // ---------------- dequant groups ----------------
+    // Group g takes the steps li = g, g + G, ...: it splices each step's T
+    // tiles into its TMEM slot 2g + (j & 1) (j = li / G), then every warp
+    // reports the slot written and moves on to the next step; the group's
+    // issuer warps take it from there.
     const int g = warp >> 2;
     const int quad = warp & 3;               // TMEM lanes 32*quad .. 32*quad+31
     const int r = quad * 32 + lane;          // weight row within the tile
-    // issuer index of this warp in its group (-1: not an issuer); the issuers
-    // of the three groups sit on different SM sub-partitions
-    const int iss = (quad == g) ? 0 : (S::kIss == 2 && quad == ((g + 2) & 3)) ? 1 : -1;
-    const bool issuer = iss >= 0;
-    constexpr int kSlice = 4 / S::kIss;      // k-slices of a tile per issuer
-    const int kk0 = (iss < 0 ? 0 : iss) * kSlice;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    bool ok = true;
+    int j = 0;                               // this group's steps so far
+    for (int li = g; li < n_local; li += S::kGroups, ++j) {
+      const int sw = li % kSW;
+      const int slot = 2 * g + (j & 1);           // also the x stage
+      ok = warp_wait(smem_u32(&wfull[sw]), (li / kSW) & 1, s_abort) && ok;
+      if (j >= 2) ok = warp_wait(smem_u32(&slotfree[slot]), ((j >> 1) - 1) & 1, s_abort) && ok;
+      tc_fence_after();
+      if (ok) {
+        const uint8_t* wst = smem + S::kWOff + sw * S::kWStage;
+        static_assert(S::kTMax == 2, "two tiles per step at most");
+        // both tiles' words first, so the second tile's loads overlap the
+        // first tile's rebuild
+        uint32_t F0[Fm::kRowWords], F1[Fm::kRowWords], w[32];
+        Fm::load(wst, r, F0);
+        if (T > 1) Fm::load(wst + Fm::kTileBytes, r, F1);
+        Fm::rebuild(F0, w);
+        tmem_st_32x32b_x32(tmem + lane_base + slot * S::kSlotCols, w);
+        if (T > 1) {
+          Fm::rebuild(F1, w);
+          tmem_st_32x32b_x32(tmem + lane_base + slot * S::kSlotCols + 32, w);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&wempty[sw]));   // smem fragments read
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&slotready[slot]));
+    }
+  } else if (warp >= S::kIssWarp && warp < S::kIssWarp + S::kGroups * S::kIss) {
+    // ---------------- MMA issuers, kIss per group ----------------
+    const int ii = warp - S::kIssWarp;
+    const int g = ii / S::kIss;
+    const int iss = ii - g * S::kIss;
+    constexpr int kSlice = 4 / S::kIss;      // k-slices of a tile per issuer
+    const int kk0 = iss * kSlice;
     constexpr uint32_t idesc = idesc_f16_f32(128, NCOL);
     bool ok = true;
     int j = 0;                               // this group's steps so far
@@ -241,72 +286,46 @@ __global__ void __launch_bounds__(DecodeShape<NCOL, F>::kThreads, 1)
       int a, b;
       segment_range(sg, tile_first, s0, KS, n_local, &a, &b);
       const int set = sg % S::kSets;
-      const uint32_t d_tmem = tmem + S::kDCol + ((set * S::kGroups + g) * S::kIss + (iss < 0 ? 0 : iss)) * NCOL;
+      const uint32_t d_tmem = tmem + S::kDCol + ((set * S::kGroups + g) * S::kIss + iss) * NCOL;
       // The accumulators of this set were last used kSets segments ago: the
       // epilogue must have read them before the first MMA or arrival.
-      if (issuer && sg >= S::kSets)
-        ok = warp_wait(smem_u32(&dempty[set]), ((sg / S::kSets) - 1) & 1, s_abort) && ok;
+      if (sg >= S::kSets) ok = warp_wait(smem_u32(&dempty[set]), ((sg / S::kSets) - 1) & 1, s_abort) && ok;
       bool first = true;
       for (int li = group_first(g, a, S::kGroups); li <= b; li += S::kGroups, ++j) {
-        const int sw = li % kSW;
-        const int sx = li % kRX;
         const int slot = 2 * g + (j & 1);
-        ok = warp_wait(smem_u32(&wfull[sw]), (li / kSW) & 1, s_abort) && ok;
-        if (j >= 2) ok = warp_wait(smem_u32(&slotfree[slot]), ((j >> 1) - 1) & 1, s_abort) && ok;
-        tc_fence_after();
-        if (ok) {
-          const uint8_t* wst = smem + S::kWOff + sw * S::kWStage;
-          for (int t = 0; t < T; ++t) {
-            uint32_t Fw[Fm::kRowWords], w[32];
-            Fm::load(wst + t * Fm::kTileBytes, r, Fw);
-            Fm::rebuild(Fw, w);
-            tmem_st_32x32b_x32(tmem + lane_base + slot * S::kSlotCols + t * 32, w);
-          }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&wempty[sw]));   // smem fragments read
-        tmem_wait_st();
-        tc_fence_before();
-        named_bar_sync(1 + g, 128);                          // the slot is written by all four warps
-        if (issuer) {
-          ok = warp_wait(smem_u32(&xfull[sx]), (li / kRX) & 1, s_abort) && ok;
-          if (lane == 0) {
-            tc_fence_after();
-            if (ok) {
-              const uint64_t bdesc0 = smem_desc_sw128(smem_u32(smem + sx * S::kXStage));
-              const uint32_t a0 = tmem + slot * S::kSlotCols;
-              for (int t = 0; t < T; ++t) {
-                const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(t * (S::kXTile >> 4));
+        ok = warp_wait(smem_u32(&slotready[slot]), (j >> 1) & 1, s_abort) && ok;
+        ok = warp_wait(smem_u32(&xfull[slot]), (j >> 1) & 1, s_abort) && ok;
+        if (lane == 0) {
+          tc_fence_after();
+          if (ok) {
+            const uint64_t bdesc0 = smem_desc_sw128(smem_u32(smem + slot * S::kXStage));
+            const uint32_t a0 = tmem + slot * S::kSlotCols;
+            for (int t = 0; t < T; ++t) {
+              const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(t * (S::kXTile >> 4));
 #pragma unroll
-                for (int q = 0; q < kSlice; ++q) {
-                  const int kk = kk0 + q;
-                  mma_f16_ts(d_tmem, a0 + t * 32 + kk * 8, bdesc + static_cast<uint64_t>(kk * 2), idesc,
-                             (first && t == 0 && q == 0) ? 0u : 1u);
-                }
+              for (int q = 0; q < kSlice; ++q) {
+                const int kk = kk0 + q;
+                mma_f16_ts(d_tmem, a0 + t * 32 + kk * 8, bdesc + static_cast<uint64_t>(kk * 2), idesc,
+                           (first && t == 0 && q == 0) ? 0u : 1u);
               }
             }
-            tc_commit(smem_u32(&slotfree[slot]));
-            tc_commit(smem_u32(&xempty[sx]));
           }
-          __syncwarp();
-        }
-        first = false;
-      }
-      // One arrival per group and segment: the commit covers this group's
-      // MMAs into the set; a group with no step in the segment just arrives.
-      if (issuer) {
-        if (lane == 0) {
-          if (!first) tc_commit(smem_u32(&dfull[set]));
-          else mbar_arrive(smem_u32(&dfull[set]));
+          tc_commit(smem_u32(&slotfree[slot]));
         }
         __syncwarp();
+        first = false;
       }
-    }
-    if (issuer) {
-      if (lane == 0) tc_commit(smem_u32(done));
+      // One arrival per issuer and segment: the commit covers this issuer's
+      // MMAs into the set; an issuer with no step in the segment just arrives.
+      if (lane == 0) {
+        if (!first) tc_commit(smem_u32(&dfull[set]));
+        else mbar_arrive(smem_u32(&dfull[set]));
+      }
       __syncwarp();
-      warp_wait(smem_u32(done), 0, s_never);
     }
+    if (lane == 0) tc_commit(smem_u32(done));
+    __syncwarp();
+    warp_wait(smem_u32(done), 0, s_never);
   } else if (warp >= S::kEpiWarp && warp < S::kEpiWarp + 4) {
     // ---------------- epilogue warpgroup: segments in order ----------------
     // A split row tile is finished by its first CTA c_lo, which reaches the
