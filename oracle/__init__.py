@@ -77,6 +77,16 @@ def _load():
             for f in ("oracle_fpx_codes", "oracle_fpx_decode_table", "oracle_fpx_round", "oracle_fpx_quantize",
                       "oracle_fpx_prepack", "oracle_fpx_unpack", "oracle_fpx_dequant", "oracle_fpx_linear"):
                 getattr(lib, f).restype = ctypes.c_int
+            lib.oracle_s24_quantize.argtypes = [P, I64, I64, P, P, P]
+            lib.oracle_s24_packed_bytes.argtypes = [I64, I64]
+            lib.oracle_s24_packed_bytes.restype = I64
+            lib.oracle_s24_prepack.argtypes = [P, P, I64, I64, P]
+            lib.oracle_s24_unpack.argtypes = [P, I64, I64, P, P]
+            lib.oracle_s24_dequant.argtypes = [P, P, I64, I64, P]
+            lib.oracle_s24_linear.argtypes = [P, P, P, P, I64, I64, I64, P]
+            for f in ("oracle_s24_quantize", "oracle_s24_prepack", "oracle_s24_unpack", "oracle_s24_dequant",
+                      "oracle_s24_linear"):
+                getattr(lib, f).restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -255,4 +265,73 @@ def fpx_linear(fmt: int, x16: np.ndarray, codes: np.ndarray, scales: np.ndarray)
     st = _load().oracle_fpx_linear(int(fmt), _ptr(x16), _ptr(codes), _ptr(scales), M, N, K, _ptr(y))
     if st != OK:
         raise OracleError(st, "fpx_linear")
+    return y
+
+
+# ---- 2:4 sparse INT4 (Sparse-Marlin): kept codes, their positions, row scales ----
+
+
+def s24_quantize(W: np.ndarray):
+    """W [N,K] fp32 -> (q [N,K/2] int8, pos [N,K/2] uint8, scales [N] fp16 bits)."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    N, K = W.shape
+    q = np.zeros((N, K // 2), dtype=np.int8)
+    pos = np.zeros((N, K // 2), dtype=np.uint8)
+    scales = np.zeros(N, dtype=np.uint16)
+    st = _load().oracle_s24_quantize(_ptr(W), N, K, _ptr(q), _ptr(pos), _ptr(scales))
+    if st != OK:
+        raise OracleError(st, "s24_quantize")
+    return q, pos, scales
+
+
+def s24_packed_bytes(N: int, K: int) -> int:
+    return int(_load().oracle_s24_packed_bytes(N, K))
+
+
+def s24_prepack(q: np.ndarray, pos: np.ndarray) -> np.ndarray:
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    pos = np.ascontiguousarray(pos, dtype=np.uint8)
+    N, K2 = q.shape
+    out = np.zeros(s24_packed_bytes(N, 2 * K2), dtype=np.uint8)
+    st = _load().oracle_s24_prepack(_ptr(q), _ptr(pos), N, 2 * K2, _ptr(out))
+    if st != OK:
+        raise OracleError(st, "s24_prepack")
+    return out
+
+
+def s24_unpack(packed: np.ndarray, N: int, K: int):
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    q = np.zeros((N, K // 2), dtype=np.int8)
+    pos = np.zeros((N, K // 2), dtype=np.uint8)
+    st = _load().oracle_s24_unpack(_ptr(packed), N, K, _ptr(q), _ptr(pos))
+    if st != OK:
+        raise OracleError(st, "s24_unpack")
+    return q, pos
+
+
+def s24_dequant(packed: np.ndarray, scales, N: int, K: int) -> np.ndarray:
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    out = np.zeros((N, K), dtype=np.uint16)
+    sp = None
+    if scales is not None:
+        scales = np.ascontiguousarray(scales, dtype=np.uint16)
+        sp = _ptr(scales)
+    st = _load().oracle_s24_dequant(_ptr(packed), sp, N, K, _ptr(out))
+    if st != OK:
+        raise OracleError(st, "s24_dequant")
+    return out
+
+
+def s24_linear(x16: np.ndarray, q: np.ndarray, pos: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    x16 = np.ascontiguousarray(x16, dtype=np.uint16)
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    pos = np.ascontiguousarray(pos, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint16)
+    M, K = x16.shape
+    N = q.shape[0]
+    assert q.shape == (N, K // 2) and pos.shape == q.shape and scales.shape == (N,)
+    y = np.zeros((M, N), dtype=np.uint16)
+    st = _load().oracle_s24_linear(_ptr(x16), _ptr(q), _ptr(pos), _ptr(scales), M, N, K, _ptr(y))
+    if st != OK:
+        raise OracleError(st, "s24_linear")
     return y

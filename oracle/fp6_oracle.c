@@ -633,3 +633,194 @@ int oracle_fpx_linear(int fmt, const uint16_t *x, const uint8_t *codes, const ui
     free(xr);
     return ORC_OK;
 }
+
+/* ---- 2:4 sparse INT4 weights (Sparse-Marlin) --------------------------------
+ * The Sparse-Marlin post (INT4 x FP16 kernel with 2:4 sparsity) names the
+ * pieces: 4-bit weights, 2:4 sparsity with metadata giving the positions of
+ * the kept weights, quantization statistics, sparse tensor cores.  It fixes
+ * none of their details; the readings taken here are the plain ones:
+ *   pruning  in each group of 4 consecutive weights of a row (k = 4j..4j+3)
+ *            the two with the largest |w| are kept, ties going to the lower
+ *            position; the other two become zero;
+ *   scale    one fp16 scale per output row, s = fp16_rne(fp32(max|w| / 7));
+ *   codes    q = round-half-even(w / s), clamped to [-8, 7] (signed 4-bit);
+ *   value    s * q at the kept positions, 0 elsewhere.
+ * Per group the two kept codes are stored in position order with their
+ * positions i0 < i1 (2 bits each).
+ */
+
+/* Positions kept in one group of four (i0 < i1). */
+static void s24_keep(const float *w, int *i0, int *i1)
+{
+    int best = 0;
+    for (int i = 1; i < 4; ++i)
+        if (fabsf(w[i]) > fabsf(w[best])) best = i;          /* strict: ties keep the lower */
+    int second = -1;
+    for (int i = 0; i < 4; ++i) {
+        if (i == best) continue;
+        if (second < 0 || fabsf(w[i]) > fabsf(w[second])) second = i;
+    }
+    *i0 = best < second ? best : second;
+    *i1 = best < second ? second : best;
+}
+
+/* Round-half-even of v (binary64) to an integer, clamped to [-8, 7]. */
+static int s24_round(double v)
+{
+    double r = nearbyint(v);                                 /* default rounding: to nearest, ties to even */
+    if (r > 7.0) r = 7.0;
+    if (r < -8.0) r = -8.0;
+    return (int)r;
+}
+
+/* W [N,K] fp32 -> q [N,K/2] (int8, kept codes in position order),
+ * pos [N,K/2] (their positions 0..3 within the group), scales [N] (fp16 bits).
+ * K must be a multiple of 4. */
+int oracle_s24_quantize(const float *W, int64_t N, int64_t K, int8_t *q, uint8_t *pos, uint16_t *scales)
+{
+    if (N < 0 || K < 0) return ORC_ERR_INVALID_ARG;
+    if (K % 4) return ORC_ERR_UNSUPPORTED_SHAPE;
+    for (int64_t n = 0; n < N; ++n) {
+        const float *row = W + n * K;
+        float amax = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            if (!isfinite(row[k])) return ORC_ERR_NONFINITE;
+            float a = fabsf(row[k]);
+            if (a > amax) amax = a;
+        }
+        double s = 0.0;
+        if (amax == 0.0f) {
+            scales[n] = 0;
+        } else {
+            volatile float s32 = amax / 7.0f;                /* IEEE fp32 division */
+            uint16_t s16 = oracle_f64_to_f16_rne((double)s32);
+            if ((s16 & 0x7FFFu) >= 0x7C00u || (s16 & 0x7FFFu) == 0) return ORC_ERR_SCALE_RANGE;
+            scales[n] = s16;
+            s = oracle_f16_to_f64(s16);
+        }
+        for (int64_t j = 0; j < K / 4; ++j) {
+            int i0, i1;
+            s24_keep(row + 4 * j, &i0, &i1);
+            int64_t o = n * (K / 2) + 2 * j;
+            pos[o] = (uint8_t)i0;
+            pos[o + 1] = (uint8_t)i1;
+            q[o] = (int8_t)(s > 0.0 ? s24_round((double)row[4 * j + i0] / s) : 0);
+            q[o + 1] = (int8_t)(s > 0.0 ? s24_round((double)row[4 * j + i1] / s) : 0);
+        }
+    }
+    return ORC_OK;
+}
+
+/* Packed size: 3/8 byte per weight (two 4-bit codes and two 2-bit positions
+ * per four weights). */
+int64_t oracle_s24_packed_bytes(int64_t N, int64_t K)
+{
+    return N * K / 8 * 3;
+}
+
+/* Packed layout: tiles of 128 rows x 64 columns, 3072 bytes each, stored
+ * like the other formats' tiles (column-tile index fastest).  Row r of a tile
+ * owns four code words V_w at byte r*16 + 4w and two position words P_h at
+ * byte 2048 + r*8 + 4h.  Group j (0..15) of the tile row: its codes in byte
+ * j%4 of V_{j/4} (first kept code in the low nibble, second in the high
+ * nibble, 4-bit two's complement), its positions in bits 4(j%8)..4(j%8)+3 of
+ * P_{j/8} (i0 in the low two bits, i1 in the next two).  Words are
+ * little-endian. */
+static inline int64_t s24_tile_base(int64_t n, int64_t k, int64_t K)
+{
+    return ((n / 128) * (K / 64) + (k / 64)) * 3072;
+}
+
+int oracle_s24_prepack(const int8_t *q, const uint8_t *pos, int64_t N, int64_t K, uint8_t *packed)
+{
+    if (N < 0 || K < 0) return ORC_ERR_INVALID_ARG;
+    if (N % 128 || K % 64) return ORC_ERR_UNSUPPORTED_SHAPE;
+    memset(packed, 0, (size_t)(N * K / 8 * 3));
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t g = 0; g < K / 4; ++g) {                /* group g of the row: columns 4g..4g+3 */
+            int64_t base = s24_tile_base(n, 4 * g, K);
+            int r = (int)(n % 128), j = (int)(g % 16);
+            int64_t o = n * (K / 2) + 2 * g;
+            uint8_t codes = (uint8_t)((q[o] & 0xF) | ((q[o + 1] & 0xF) << 4));
+            packed[base + r * 16 + 4 * (j / 4) + (j % 4)] = codes;
+            uint8_t meta = (uint8_t)((pos[o] & 3) | ((pos[o + 1] & 3) << 2));
+            int bit = 4 * (j % 8);
+            packed[base + 2048 + r * 8 + 4 * (j / 8) + bit / 8] |= (uint8_t)(meta << (bit % 8));
+        }
+    return ORC_OK;
+}
+
+int oracle_s24_unpack(const uint8_t *packed, int64_t N, int64_t K, int8_t *q, uint8_t *pos)
+{
+    if (N < 0 || K < 0) return ORC_ERR_INVALID_ARG;
+    if (N % 128 || K % 64) return ORC_ERR_UNSUPPORTED_SHAPE;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t g = 0; g < K / 4; ++g) {
+            int64_t base = s24_tile_base(n, 4 * g, K);
+            int r = (int)(n % 128), j = (int)(g % 16);
+            int64_t o = n * (K / 2) + 2 * g;
+            uint8_t codes = packed[base + r * 16 + 4 * (j / 4) + (j % 4)];
+            int lo = codes & 0xF, hi = codes >> 4;
+            q[o] = (int8_t)(lo >= 8 ? lo - 16 : lo);
+            q[o + 1] = (int8_t)(hi >= 8 ? hi - 16 : hi);
+            int bit = 4 * (j % 8);
+            uint8_t meta = (uint8_t)((packed[base + 2048 + r * 8 + 4 * (j / 8) + bit / 8] >> (bit % 8)) & 0xF);
+            pos[o] = (uint8_t)(meta & 3);
+            pos[o + 1] = (uint8_t)(meta >> 2);
+        }
+    return ORC_OK;
+}
+
+/* Dense fp16 weights: fp16_rne(s * q) at the kept positions (fp16(q) without
+ * scales), +0 elsewhere. */
+int oracle_s24_dequant(const uint8_t *packed, const uint16_t *scales, int64_t N, int64_t K, uint16_t *W16)
+{
+    if (N < 0 || K < 0) return ORC_ERR_INVALID_ARG;
+    if (N % 128 || K % 64) return ORC_ERR_UNSUPPORTED_SHAPE;
+    int8_t *q = (int8_t *)malloc((size_t)(N * K / 2) + 1);
+    uint8_t *pos = (uint8_t *)malloc((size_t)(N * K / 2) + 1);
+    if (!q || !pos) {
+        free(q);
+        free(pos);
+        return ORC_ERR_INVALID_ARG;
+    }
+    oracle_s24_unpack(packed, N, K, q, pos);
+    memset(W16, 0, sizeof(uint16_t) * (size_t)(N * K));
+    for (int64_t n = 0; n < N; ++n) {
+        double s = scales ? oracle_f16_to_f64(scales[n]) : 1.0;
+        for (int64_t g = 0; g < K / 4; ++g)
+            for (int a = 0; a < 2; ++a) {
+                int64_t o = n * (K / 2) + 2 * g + a;
+                W16[n * K + 4 * g + pos[o]] = oracle_f64_to_f16_rne(s * (double)q[o]);
+            }
+    }
+    free(q);
+    free(pos);
+    return ORC_OK;
+}
+
+/* y[M,N] = fp16_rne( sum_k x[m,k] * s_n * v[n,k] ), v the dense code values
+ * (q at kept positions, 0 elsewhere), summed in binary64. */
+int oracle_s24_linear(const uint16_t *x, const int8_t *q, const uint8_t *pos, const uint16_t *scales,
+                      int64_t M, int64_t N, int64_t K, uint16_t *y)
+{
+    if (M < 0 || N < 0 || K < 0) return ORC_ERR_INVALID_ARG;
+    if (K % 4) return ORC_ERR_UNSUPPORTED_SHAPE;
+    double *xr = (double *)malloc(sizeof(double) * (size_t)(K > 0 ? K : 1));
+    if (!xr) return ORC_ERR_INVALID_ARG;
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t k = 0; k < K; ++k) xr[k] = oracle_f16_to_f64(x[m * K + k]);
+        for (int64_t n = 0; n < N; ++n) {
+            double s = oracle_f16_to_f64(scales[n]);
+            double acc = 0.0;
+            for (int64_t g = 0; g < K / 4; ++g)
+                for (int a = 0; a < 2; ++a) {
+                    int64_t o = n * (K / 2) + 2 * g + a;
+                    acc += xr[4 * g + pos[o]] * (s * (double)q[o]);
+                }
+            y[m * N + n] = oracle_f64_to_f16_rne(acc);
+        }
+    }
+    free(xr);
+    return ORC_OK;
+}
