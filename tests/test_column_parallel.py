@@ -52,6 +52,21 @@ def test_packed_slice_is_the_packing_of_the_row_slice(orc, world):
         assert np.array_equal(s, scales[n0:n1])
 
 
+@pytest.mark.parametrize("fmt", [0, 1, 2, 3])
+def test_packed_slice_other_formats(orc, fmt):
+    """The same for the other weight formats: a rank's byte range of the full
+    packed buffer is the packing of its rows alone."""
+    N, K, world = 640, 128, 3
+    ncodes = orc.fpx_codes(fmt)
+    codes = np.random.default_rng(fmt).integers(0, ncodes, size=(N, K)).astype(np.uint8)
+    packed = orc.fpx_prepack(fmt, codes)
+    scales = np.arange(N, dtype=np.uint16)
+    for r in range(world):
+        p, s, n0, n1 = cp.shard_packed(packed, scales, N, K, world, r, fmt)
+        assert np.array_equal(p, orc.fpx_prepack(fmt, codes[n0:n1]))
+        assert np.array_equal(s, scales[n0:n1])
+
+
 def _free_port():
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))

@@ -14,9 +14,15 @@ every step of the product runs in libfp6.
 """
 from __future__ import annotations
 
+from fractions import Fraction
+
 from . import _lib
 
 TILE_ROWS = 128
+
+# bytes per weight of each packed format (None = FP6 e3m2, as fp6_*)
+_BYTES_PER_WEIGHT = {None: Fraction(3, 4), 0: Fraction(3, 4), 1: Fraction(3, 4), 2: Fraction(1, 2),
+                     3: Fraction(5, 8)}
 
 
 def shard_rows(N: int, world: int, rank: int) -> tuple[int, int]:
@@ -33,18 +39,23 @@ def shard_rows(N: int, world: int, rank: int) -> tuple[int, int]:
     return t0 * TILE_ROWS, t1 * TILE_ROWS
 
 
-def packed_range(K: int, n0: int, n1: int) -> tuple[int, int]:
+def packed_range(K: int, n0: int, n1: int, fmt=None) -> tuple[int, int]:
     """Byte range [b0, b1) of rows [n0, n1) inside the packed buffer of an
-    N x K weight (0.75 bytes per weight, row tiles stored one after another)."""
+    N x K weight: every format stores its 128-row tiles one after another, so
+    whole row tiles are one contiguous range (0.75 bytes per weight for the
+    6-bit formats, 0.625 for FP5, 0.5 for FP4)."""
     if n0 % TILE_ROWS or n1 % TILE_ROWS or K % 64:
         raise ValueError("rows must be whole 128-row tiles and K a multiple of 64")
-    return n0 * K * 3 // 4, n1 * K * 3 // 4
+    if fmt not in _BYTES_PER_WEIGHT:
+        raise ValueError(f"unknown format {fmt!r}")
+    b = _BYTES_PER_WEIGHT[fmt]
+    return int(n0 * K * b), int(n1 * K * b)
 
 
-def shard_packed(packed, scales, N: int, K: int, world: int, rank: int):
+def shard_packed(packed, scales, N: int, K: int, world: int, rank: int, fmt=None):
     """This rank's (packed, scales, n0, n1) views of a full packed weight."""
     n0, n1 = shard_rows(N, world, rank)
-    b0, b1 = packed_range(K, n0, n1)
+    b0, b1 = packed_range(K, n0, n1, fmt)
     return packed[b0:b1], scales[n0:n1], n0, n1
 
 
@@ -68,13 +79,15 @@ def gather_columns(y_local, N: int, group=None):
 
 class ColumnParallelFP6Linear:
     """y = x . (scale (.) decode(W))^T with W's rows split across the ranks of
-    `group` (torch.distributed, NCCL on GPUs).  Construct it on every rank
+    `group` (torch.distributed, NCCL on GPUs); `fmt` selects the weight format
+    as in linear().  Construct it on every rank
     from the full packed weight (only this rank's slice is kept on its GPU) or
     from an already sliced one (pass shard=True)."""
 
-    def __init__(self, packed, scales, N: int, K: int, group=None, shard: bool = False):
+    def __init__(self, packed, scales, N: int, K: int, group=None, shard: bool = False, fmt=None):
         import torch.distributed as dist
         self.group = group
+        self.fmt = fmt
         self.world = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
         self.N, self.K = N, K
@@ -82,7 +95,7 @@ class ColumnParallelFP6Linear:
         if shard:
             self.packed, self.scales = packed, scales
         else:
-            self.packed, self.scales, _, _ = shard_packed(packed, scales, N, K, self.world, self.rank)
+            self.packed, self.scales, _, _ = shard_packed(packed, scales, N, K, self.world, self.rank, fmt)
             self.packed = self.packed.contiguous().clone()
             self.scales = self.scales.contiguous().clone()
 
@@ -90,7 +103,7 @@ class ColumnParallelFP6Linear:
         """This rank's output columns y[:, n0:n1]."""
         from . import linear
         _lib.load()                          # fail loudly without the CUDA library
-        return linear(x, self.packed, self.scales, self.n1 - self.n0, self.K, out=out)
+        return linear(x, self.packed, self.scales, self.n1 - self.n0, self.K, out=out, fmt=self.fmt)
 
     def __call__(self, x, gather: bool = True):
         y = self.local(x)
