@@ -207,6 +207,25 @@ def test_workload_sampled(fp6, orc, cfg, li, lname, N, K, Ms, outliers):
         parity.assert_close(y[np.ix_(toks, rows)], ref, f"{lname} N={N} K={K} M={M}")
 
 
+@pytest.mark.parametrize("N,K,M", [(18944, 128, 300), (18944, 128, 1100), (148 * 128 * 2, 192, 257)])
+def test_wave_schedule(fp6, orc, N, K, M):
+    """Shapes whose tiles fill whole waves of 148 CTAs (148 or 296 row tiles
+    times 2 or 5 token tiles, the last token tile ragged), through the general
+    kernel; checked on sampled rows (two whole 128-row tiles and random rows)
+    and sampled tokens."""
+    from weight_only_quantized_fp6_b200 import inputs
+    W = inputs.weights(N + K, N, K)
+    x = inputs.activations(M, M, K)
+    codes, scales, packed = gpu_layer(fp6, W)
+    y = bits16(fp6.linear(as_f16(x), packed, scales, N, K))
+    rng = np.random.default_rng(N + M)
+    rows = parity.sample_rows(N, rng)
+    toks = parity.sample_tokens(M, rng, limit=48)
+    codes_o, scales_o = orc.quantize(W[rows])
+    ref = orc.linear(x[toks], codes_o, scales_o, nthreads=16)
+    parity.assert_close(y[np.ix_(toks, rows)], ref, f"wave N={N} K={K} M={M}")
+
+
 def test_workspace_reused_across_shapes(fp6, orc):
     """One workspace serves a sequence of problems of different sizes: the
     counters left by each call (and the partials it wrote) never disturb the
