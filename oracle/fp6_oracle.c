@@ -37,6 +37,11 @@
  *                       e2m3 values), round trips, independent readers of the
  *                       FP4 and FP5 layouts, one-hot probes, exact rational dot
  *                       products
+ *   s24_* (2:4 sparse INT4)
+ *                       pinned: properties that fix the kept pair uniquely,
+ *                       brute-force rounding and exact ties, representable
+ *                       round trips, an independent layout reader, one-hot
+ *                       probes, dense dequant, exact rational dot products
  */
 #include <math.h>
 #include <stdint.h>
