@@ -186,7 +186,7 @@ def oracle_workload(rows: int):
     """Codes/scales of the first `rows` weight rows and the activations, from the oracle."""
     import oracle
     from weight_only_quantized_fp6_b200 import inputs
-    wseed = inputs.weight_seed(2, 0)
+    wseed = inputs.weight_seed("llama70b_o_decode", 0)
     W = inputs.weights(wseed, N_DIM, K_DIM, rows=range(rows))
     codes, scales = oracle.quantize(W)
     xs = {M: inputs.activations(inputs.activation_seed(wseed, M), M, K_DIM) for M in MS}
@@ -340,7 +340,7 @@ def run_fp6(args, world, rank, local):
     l2 = getattr(props, "L2_cache_size", 126 * 1024 * 1024)
 
     # weights: seeded N(0, 0.02), quantized and packed by the library
-    wseed = inputs.weight_seed(2, rank)
+    wseed = inputs.weight_seed("llama70b_o_decode", rank)
     W = inputs.weights_parallel(wseed, N_DIM, K_DIM)
     layer = fp6.FP6Linear.from_float(torch.from_numpy(W).to(dev))
     del W
@@ -550,8 +550,8 @@ def run_sweep(args):
     ws = fp6.Workspace(dev)
     fmt, bpw = FORMAT_CODE[args.fmt], FORMAT_BYTES[args.fmt]
     rows = []
-    for cfg in (2, 3, 4, 5):
-        spec = inputs.CONFIGS[cfg]
+    for wname in ("llama70b_o_decode", "llama70b_all", "opt30b", "prefill"):
+        spec = inputs.WORKLOADS[wname]
         for lname, (N, K) in spec["layers"].items():
             W = torch.randn(N, K, device=dev, generator=gen) * 0.02
             layer = fp6.FP6Linear.from_float(W, fmt=fmt)
@@ -582,7 +582,7 @@ def run_sweep(args):
                 del graph
                 t_tc = 2.0 * M * N * K / (peaks["bf16_tflops"] * 1e12)
                 t_hbm = algo_bytes(M, N, K, bpw) / (peaks["hbm_gbs"] * 1e9)
-                rows.append({"config": spec["name"], "format": args.fmt, "layer": lname, "N": N, "K": K, "M": M,
+                rows.append({"config": wname, "format": args.fmt, "layer": lname, "N": N, "K": K, "M": M,
                              "us": round(t * 1e6, 2), "weight_gbs": round(wbytes(N, K, bpw) / t / 1e9, 1),
                              "tflops": round(2.0 * M * N * K / t / 1e12, 1),
                              "bound": "tensor" if t_tc > t_hbm else "hbm",

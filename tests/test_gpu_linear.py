@@ -59,7 +59,7 @@ def run_case(fp6, orc, N, K, M, wseed, xseed, outliers=0.0):
 def test_tiny_config(fp6, orc):
     """Tiny W6A16 case: M=4, N=256, K=512, seed 0."""
     from weight_only_quantized_fp6_b200 import inputs
-    run_case(fp6, orc, 256, 512, 4, inputs.weight_seed(1, 0), inputs.activation_seed(0, 4))
+    run_case(fp6, orc, 256, 512, 4, inputs.weight_seed("tiny", 0), inputs.activation_seed(0, 4))
 
 
 @pytest.mark.parametrize("M", [1, 2, 3, 5, 15, 16, 17, 31, 33, 64, 65, 100, 128, 129, 256, 300])
@@ -175,17 +175,17 @@ def test_no_device_errors_recorded(fp6):
 # ---- the workload shapes, sampled ------------------------------------------------
 
 WORKLOADS = []
-for cfg in (2, 3, 4, 5):
-    spec = __import__("weight_only_quantized_fp6_b200.inputs", fromlist=["CONFIGS"]).CONFIGS[cfg]
+for wname in ("llama70b_o_decode", "llama70b_all", "opt30b", "prefill"):
+    spec = __import__("weight_only_quantized_fp6_b200.inputs", fromlist=["WORKLOADS"]).WORKLOADS[wname]
     for li, (lname, (N, K)) in enumerate(spec["layers"].items()):
-        WORKLOADS.append(pytest.param(cfg, li, lname, N, K, spec["M"], spec["outliers"],
-                                      id=f"{spec['name']}-{lname}"))
+        WORKLOADS.append(pytest.param(wname, li, lname, N, K, spec["M"], spec["outliers"],
+                                      id=f"{wname}-{lname}"))
 
 
-@pytest.mark.parametrize("cfg,li,lname,N,K,Ms,outliers", WORKLOADS)
-def test_workload_sampled(fp6, orc, cfg, li, lname, N, K, Ms, outliers):
+@pytest.mark.parametrize("wname,li,lname,N,K,Ms,outliers", WORKLOADS)
+def test_workload_sampled(fp6, orc, wname, li, lname, N, K, Ms, outliers):
     from weight_only_quantized_fp6_b200 import inputs
-    wseed = inputs.weight_seed(cfg, li)
+    wseed = inputs.weight_seed(wname, li)
     W = parity.gen_weights_parallel(wseed, N, K, outliers)
     codes, scales, packed = gpu_layer(fp6, W)
     del W

@@ -24,7 +24,8 @@ def test_moments_and_outliers():
 
 def test_seeds_differ():
     assert not np.array_equal(inputs.weights(1, 8, 64), inputs.weights(2, 8, 64))
-    assert inputs.activation_seed(inputs.weight_seed(2, 0), 16) == 2116
+    assert inputs.activation_seed(inputs.weight_seed("llama70b_o_decode", 0), 16) == 2116
+    assert inputs.weight_seed("tiny", 0) == 0 and inputs.weight_seed("opt30b", 3) == 4003
 
 
 def test_parallel_generation_matches():

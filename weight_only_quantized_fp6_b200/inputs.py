@@ -119,17 +119,24 @@ LLAMA70B = {"qkv": (10240, 8192), "o": (8192, 8192), "gate_up": (57344, 8192), "
 OPT30B = {"qkv": (21504, 7168), "o": (7168, 7168), "fc1": (28672, 7168), "fc2": (7168, 28672)}
 PREFILL = {"up": (28672, 8192), "down": (8192, 28672)}
 
-CONFIGS = {
-    1: {"name": "tiny", "layers": {"tiny": (256, 512)}, "M": [4], "outliers": 0.0},
-    2: {"name": "llama70b_o_decode", "layers": {"o": LLAMA70B["o"]}, "M": [1, 2, 4, 8, 16], "outliers": 0.0},
-    3: {"name": "llama70b_all", "layers": LLAMA70B, "M": [1, 4, 8, 16, 32], "outliers": 0.0},
-    4: {"name": "opt30b", "layers": OPT30B, "M": [1, 16, 64, 128], "outliers": 0.001},
-    5: {"name": "prefill", "layers": PREFILL, "M": [256, 1024, 4096], "outliers": 0.0},
+# Workloads by name: layer shapes, token counts, outlier rate, and the base of
+# the weight seeds of their layers (layer i of a workload draws its weights
+# from seed_base + i).
+WORKLOADS = {
+    "tiny": {"layers": {"tiny": (256, 512)}, "M": [4], "outliers": 0.0, "seed_base": 0},
+    "llama70b_o_decode": {"layers": {"o": LLAMA70B["o"]}, "M": [1, 2, 4, 8, 16], "outliers": 0.0,
+                          "seed_base": 2000},
+    "llama70b_all": {"layers": LLAMA70B, "M": [1, 4, 8, 16, 32], "outliers": 0.0, "seed_base": 3000},
+    "opt30b": {"layers": OPT30B, "M": [1, 16, 64, 128], "outliers": 0.001, "seed_base": 4000},
+    "prefill": {"layers": PREFILL, "M": [256, 1024, 4096], "outliers": 0.0, "seed_base": 5000},
 }
 
 
-def weight_seed(config: int, layer_index: int) -> int:
-    return 0 if config == 1 else 1000 * config + layer_index
+def weight_seed(workload: str, layer_index: int) -> int:
+    """Weight seed of layer `layer_index` of a named workload (the tiny
+    workload's single layer uses seed 0)."""
+    base = WORKLOADS[workload]["seed_base"]
+    return base if base == 0 else base + layer_index
 
 
 def activation_seed(wseed: int, M: int) -> int:
