@@ -73,13 +73,13 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _rank_main(rank, world, port, N, K, M, q):
+def _rank_main(rank, world, port, N, K, M, q, fmt=None):
     import torch.distributed as dist
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
-        _rank_work(rank, world, N, K, M, q)
+        _rank_work(rank, world, N, K, M, q, fmt)
     except Exception as e:  # report instead of leaving the parent waiting
         q.put((rank, repr(e)))
         raise
@@ -87,15 +87,22 @@ def _rank_main(rank, world, port, N, K, M, q):
         dist.destroy_process_group()
 
 
-def _rank_work(rank, world, N, K, M, q):
+def _rank_work(rank, world, N, K, M, q, fmt=None):
     import oracle
     W = inputs.weights(42, N, K)
     x = inputs.activations(43, M, K)
-    codes, scales = oracle.quantize(W)
-    packed = oracle.prepack(codes)
-    p, s, n0, n1 = cp.shard_packed(packed, scales, N, K, world, rank)
+    if fmt is None:
+        codes, scales = oracle.quantize(W)
+        packed = oracle.prepack(codes)
+    else:
+        codes, scales = oracle.fpx_quantize(fmt, W)
+        packed = oracle.fpx_prepack(fmt, codes)
+    p, s, n0, n1 = cp.shard_packed(packed, scales, N, K, world, rank, fmt)
     # this rank's output columns, from its slice of the packed weight only
-    y_local = oracle.linear(x, oracle.unpack(p, n1 - n0, K), s)
+    if fmt is None:
+        y_local = oracle.linear(x, oracle.unpack(p, n1 - n0, K), s)
+    else:
+        y_local = oracle.fpx_linear(fmt, x, oracle.fpx_unpack(fmt, p, n1 - n0, K), s)
     y = cp.gather_columns(torch.from_numpy(y_local.view(np.float16)), N)
     q.put((rank, y.numpy().view(np.uint16)))
 
@@ -118,6 +125,31 @@ def test_gloo_ranks_gather_the_full_output(orc, world, N):
     x = inputs.activations(43, M, K)
     codes, scales = orc.quantize(W)
     ref = orc.linear(x, codes, scales)
+    for r in range(world):
+        assert not isinstance(results[r], str), f"rank {r} failed: {results[r]}"
+        assert np.array_equal(results[r], ref), f"rank {r}"
+
+
+@pytest.mark.parametrize("fmt", [1, 2, 3])
+def test_gloo_ranks_gather_other_formats(orc, fmt):
+    """Two gloo ranks, each computing its columns from its byte range of a
+    packed FP6 e2m3 / FP4 / FP5 weight, gather the full oracle output."""
+    import torch.multiprocessing as mp
+    world, N, K, M = 2, 384, 192, 3
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, N, K, M, q, fmt)) for r in range(world)]
+    for pr in procs:
+        pr.start()
+    results = dict(q.get(timeout=120) for _ in range(world))
+    for pr in procs:
+        pr.join(timeout=120)
+        assert pr.exitcode == 0
+    W = inputs.weights(42, N, K)
+    x = inputs.activations(43, M, K)
+    codes, scales = orc.fpx_quantize(fmt, W)
+    ref = orc.fpx_linear(fmt, x, codes, scales)
     for r in range(world):
         assert not isinstance(results[r], str), f"rank {r} failed: {results[r]}"
         assert np.array_equal(results[r], ref), f"rank {r}"
