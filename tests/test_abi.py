@@ -34,6 +34,27 @@ def test_binding_covers_header():
     assert set(declared_functions()) == set(_lib.SIGNATURES)
 
 
+def declared_arities():
+    """Number of parameters of every function include/fp6.h declares."""
+    src = open(os.path.join(ROOT, "include", "fp6.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    out = {}
+    for m in re.finditer(r"\b(fp[6x]_[a-z_0-9]+)\s*\(([^)]*)\)\s*;", src):
+        params = m.group(2).strip()
+        out[m.group(1)] = 0 if params in ("", "void") else len(params.split(","))
+    return out
+
+
+def test_binding_argument_counts_match_header():
+    """The ctypes table passes exactly as many arguments as each C
+    declaration takes."""
+    from weight_only_quantized_fp6_b200 import _lib
+    ar = declared_arities()
+    assert set(ar) == set(_lib.SIGNATURES)
+    for name, (_, args) in _lib.SIGNATURES.items():
+        assert len(args) == ar[name], (name, len(args), ar[name])
+
+
 def test_status_strings(lib):
     from weight_only_quantized_fp6_b200 import _lib
     for code, name in _lib.STATUS.items():
