@@ -55,15 +55,22 @@ def algo_bytes(M, N, K, per_weight=0.75):
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "fp6_linear_decode_kernel_llama70b_o_proj_decode.md")
 
 
+# The device sources the decode kernel (the bench's kernel) is compiled from:
+# its own header and the headers it includes.  Its launch configuration
+# (grid = SM count, block and shared memory from DecodeShape, T = kTMax) is
+# fixed by them too.
+DECODE_KERNEL_SOURCES = ["fp6_format.cuh", "fp6_linear.cuh", "fp6_linear_decode.cuh", "ptx.cuh"]
+
+
 def kernel_source_hash() -> str:
-    """First 16 hex digits of the SHA-256 over the library's CUDA sources, sorted by name."""
+    """First 16 hex digits of the SHA-256 over the decode kernel's device
+    sources, in sorted name order."""
     import hashlib
     csrc = os.path.join(ROOT, "weight_only_quantized_fp6_b200", "csrc")
     h = hashlib.sha256()
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(f.read())
+    for name in sorted(DECODE_KERNEL_SOURCES):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 

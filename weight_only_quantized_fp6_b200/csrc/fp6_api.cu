@@ -13,6 +13,7 @@
 #include "fp6_aux_kernels.cuh"
 #include "fp6_linear.cuh"
 #include "fp6_linear_decode.cuh"
+#include "fp6_linear_wave.cuh"
 
 namespace fp6 {
 // A wait that can never complete: the mbarrier expects one arrival that no
@@ -53,7 +54,7 @@ fp6_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FP6_OK : FP6_E
 // ---- per-device cached properties ------------------------------------------
 struct DeviceInfo {
   int sms = 0;
-  bool attrs_set[4][8] = {};   // [format][kernel variant]: shared-memory limit raised
+  bool attrs_set[4][10] = {};  // [format][kernel variant]: shared-memory limit raised
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -101,6 +102,7 @@ struct Plan {
   long long total = 0;  // steps in all
   size_t counter_bytes = 0;
   size_t partial_bytes = 0;
+  bool wave = false;  // whole tiles per CTA (fp6_linear_wave.cuh) instead of stream-K ranges
 };
 
 int pick_ncol(int64_t M) {
@@ -153,6 +155,17 @@ bool make_plan(int64_t M, int64_t N, int64_t K, int sms, Plan* pl) {
   pl->grid = static_cast<int>(std::min<long long>(std::min(sms, fp6::kMaxGrid), pl->total));
   // the decode variants (NCOL <= 64) handle one token tile: NCOL >= M
   if (pl->ncol <= 64 && pl->m_tiles != 1) return false;
+  // Many tiles and a nearly full last wave (at most 5 % of the CTA-tile slots
+  // idle): whole tiles per CTA, which share weights and activations through
+  // L2; otherwise the stream-K ranges balance the work exactly.
+  if (pl->ncol > 64) {
+    const long long G = std::min(sms, fp6::kMaxGrid);
+    const long long waves = (pl->tiles + G - 1) / G;
+    if (pl->tiles >= G && waves * G * 100 <= pl->tiles * 105) {
+      pl->wave = true;
+      pl->grid = static_cast<int>(G);
+    }
+  }
   pl->counter_bytes = fp6::kCounterBytes;
   pl->partial_bytes = static_cast<size_t>(2) * pl->grid * pl->ncol * 128 * sizeof(float);
   return true;
@@ -178,6 +191,34 @@ fp6_status launch_linear(const CUtensorMap& map, const fp6::LinearParams& prm, c
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned int>(prm.grid));
   cfg.blockDim = dim3(static_cast<unsigned int>(threads));
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, map, prm) != cudaSuccess) return FP6_ERR_CUDA;
+  return cuda_status(cudaGetLastError());
+}
+
+// The wave-schedule kernel (whole tiles per CTA), launched the same way.
+template <int NCOL, Fmt F>
+fp6_status launch_wave(const CUtensorMap& map, const fp6::LinearParams& prm, cudaStream_t stream, int dev) {
+  auto kern = fp6::fp6_linear_wave_kernel<NCOL, F>;
+  const int smem = LinearShape<NCOL, F>::kSmemBytes;
+  const int idx = NCOL == 128 ? 8 : 9;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_dev[dev].attrs_set[static_cast<int>(F)][idx]) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return FP6_ERR_CUDA;
+      g_dev[dev].attrs_set[static_cast<int>(F)][idx] = true;
+    }
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned int>(prm.grid));
+  cfg.blockDim = dim3(static_cast<unsigned int>(fp6::kLinearThreads));
   cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -350,8 +391,8 @@ fp6_status linear_impl(const uint16_t* x, const void* packed, const uint16_t* sc
     case 16: return launch_decode<16, F>(map, prm, stream, dev);
     case 32: return launch_decode<32, F>(map, prm, stream, dev);
     case 64: return launch_decode<64, F>(map, prm, stream, dev);
-    case 128: return launch_linear<128, F>(map, prm, stream, dev);
-    default: return launch_linear<256, F>(map, prm, stream, dev);
+    case 128: return pl.wave ? launch_wave<128, F>(map, prm, stream, dev) : launch_linear<128, F>(map, prm, stream, dev);
+    default: return pl.wave ? launch_wave<256, F>(map, prm, stream, dev) : launch_linear<256, F>(map, prm, stream, dev);
   }
 }
 
