@@ -180,6 +180,13 @@ fp6_status fp6_linear_noalloc(const uint16_t *x, const void *packed, const uint1
  * Returns FP6_OK or an argument error. */
 fp6_status fp6_linear_plan(int64_t M, int64_t N, int64_t K, int64_t out[5]);
 
+/* The same plan for a device with `sms` multiprocessors, computed on the host
+ * alone (no CUDA call; for tests and capacity planning):
+ * out[0..4] as fp6_linear_plan, out[5] = 64-column tiles per step (T),
+ * out[6] = 1 when the wave-schedule kernel (whole tiles per CTA) runs, else 0.
+ * Returns FP6_OK or an argument error (sms <= 0 is FP6_ERR_INVALID_ARG). */
+fp6_status fp6_linear_plan_for_sms(int64_t M, int64_t N, int64_t K, int sms, int64_t out[7]);
+
 /*
  * Other float formats -- the FP6-LLM pages present the design as one for
  * float weights of several bit widths (TC-FPx: "x" bits); these entry points

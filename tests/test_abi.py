@@ -137,3 +137,56 @@ def test_oracle_is_not_linked_into_the_library():
     for name in os.listdir(pkg):
         if name.endswith(".py"):
             assert "import oracle" not in open(os.path.join(pkg, name)).read(), name
+
+
+def plan(lib, M, N, K, sms=148):
+    out = (ctypes.c_int64 * 7)()
+    assert lib.fp6_linear_plan_for_sms(M, N, K, sms, out) == 0
+    return {"ncol": out[0], "stages": out[1], "grid": out[2], "tiles": out[3], "total": out[4], "T": out[5],
+            "wave": out[6]}
+
+
+def test_plan_token_tiles_and_steps(lib):
+    """Token-tile width by M (16, 32, 64 for the decode kernel; 128, 256
+    beyond), the widest step that divides K / 64, and a grid of at most one
+    CTA per SM and per step."""
+    for M, ncol in [(1, 16), (16, 16), (17, 32), (32, 32), (33, 64), (64, 64), (65, 128), (128, 128),
+                    (129, 256), (4096, 256)]:
+        assert plan(lib, M, 8192, 8192)["ncol"] == ncol, M
+    assert plan(lib, 1, 8192, 8192)["T"] == 2
+    assert plan(lib, 1, 8192, 64 * 3)["T"] == 1            # three column tiles: odd, one tile per step
+    p = plan(lib, 1, 128, 64)
+    assert p["total"] == 1 and p["grid"] == 1               # never more CTAs than steps
+    p = plan(lib, 1, 8192, 8192)
+    assert p["grid"] == 148 and p["tiles"] == 64 and p["total"] == 64 * 64
+    assert plan(lib, 16, 8192, 8192, sms=132)["grid"] == 132
+
+
+def test_plan_wave_schedule_rule(lib):
+    """Whole tiles per CTA only with at least as many tiles as SMs and a last
+    wave at least 95 % full; every CTA then has a tile."""
+    cases = [
+        (4096, 28672, 8192, 1),    # 3584 tiles: 25 waves, 3.3 % idle
+        (4096, 8192, 28672, 1),    # 1024 tiles: 7 waves, 1.4 % idle
+        (4096, 21504, 7168, 1),    # 2688 tiles: 19 waves, 4.6 % idle
+        (1024, 28672, 8192, 0),    # 896 tiles: 7 waves, 13.5 % idle
+        (1024, 8192, 28672, 0),    # 256 tiles: 2 waves
+        (256, 28672, 8192, 0),     # 224 tiles
+        (300, 18944, 128, 1),      # 296 tiles: 2 waves, exactly full
+        (16, 57344, 8192, 0),      # decode kernel: never
+    ]
+    for M, N, K, wave in cases:
+        p = plan(lib, M, N, K)
+        assert p["wave"] == wave, (M, N, K)
+        if wave:
+            assert p["grid"] == 148 and p["tiles"] >= 148
+            waves = -(-p["tiles"] // 148)
+            assert waves * 148 * 100 <= p["tiles"] * 105
+
+
+def test_plan_for_sms_rejects_bad_arguments(lib):
+    out = (ctypes.c_int64 * 7)()
+    assert lib.fp6_linear_plan_for_sms(1, 8192, 8192, 0, out) == 1
+    assert lib.fp6_linear_plan_for_sms(-1, 8192, 8192, 148, out) == 1
+    assert lib.fp6_linear_plan_for_sms(1, 100, 8192, 148, out) == 2
+    assert lib.fp6_linear_plan_for_sms(1, 8192, 8192, 148, None) == 1

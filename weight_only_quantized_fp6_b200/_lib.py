@@ -34,6 +34,7 @@ SIGNATURES = {
     "fp6_linear": (_ST, [_P, _P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     "fp6_get_device_status": (_ST, [_P]),
     "fp6_linear_plan": (_ST, [_I64, _I64, _I64, ctypes.POINTER(_I64)]),
+    "fp6_linear_plan_for_sms": (_ST, [_I64, _I64, _I64, ctypes.c_int, ctypes.POINTER(_I64)]),
     "fp6_linear_noalloc": (_ST, [_P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "fp6_selftest_wait_timeout": (_ST, [_P]),
     "fpx_packed_bytes": (_SZ, [_ST, _I64, _I64]),

@@ -454,6 +454,24 @@ fp6_status fp6_linear_plan(int64_t M, int64_t N, int64_t K, int64_t out[5]) {
   return FP6_OK;
 }
 
+fp6_status fp6_linear_plan_for_sms(int64_t M, int64_t N, int64_t K, int sms, int64_t out[7]) {
+  if (!out) return FP6_ERR_INVALID_ARG;
+  fp6_status st = check_shape(N, K);
+  if (st != FP6_OK) return st;
+  if (M < 0 || sms <= 0) return FP6_ERR_INVALID_ARG;
+  if (M > INT32_MAX) return FP6_ERR_UNSUPPORTED_SHAPE;
+  Plan pl;
+  make_plan(M, N, K, sms, &pl);
+  out[0] = pl.ncol;
+  out[1] = pl.stages;
+  out[2] = pl.grid;
+  out[3] = pl.tiles;
+  out[4] = pl.total;
+  out[5] = pl.T;
+  out[6] = pl.wave ? 1 : 0;
+  return FP6_OK;
+}
+
 size_t fp6_linear_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   if (check_shape(N, K) != FP6_OK || M < 0 || M > INT32_MAX) return 0;
   int dev = 0;
