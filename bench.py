@@ -361,30 +361,32 @@ def run_fp6(args, world, rank, local):
     ws.get(max(fp6.workspace_bytes(M, N_DIM, K_DIM) for M in MS))
 
     stream = torch.cuda.Stream(device=dev)
-    # One CUDA graph per rotation offset, holding the step's 5 launches back to
-    # back (kernel nodes only, so consecutive launches keep their programmatic
-    # dependent-launch overlap).
-    n_graphs = copies
-    graphs = []
+    # The timed steps are captured in one CUDA graph, as a serving engine runs
+    # a decode step: each step's 5 launches back to back, every launch on the
+    # next packed copy (kernel nodes only, so consecutive launches keep their
+    # programmatic dependent-launch overlap, across step boundaries too).
+    # Replaying it once runs exactly args.steps steps; a second graph of
+    # args.warmup steps is the warm-up.
+    def capture(n_steps):
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for s in range(n_steps):
+                for i, M in enumerate(MS):
+                    fp6.linear(xs[M], packs[(s * len(MS) + i) % copies], scales, N_DIM, K_DIM,
+                               out=ys[M], workspace=ws)
+        return graph
+
     with torch.cuda.stream(stream):
         for M in MS:  # eager warm-up (sets kernel attributes before capture)
             fp6.linear(xs[M], packs[0], scales, N_DIM, K_DIM, out=ys[M], workspace=ws)
         stream.synchronize()
-        for g in range(n_graphs):
-            graph = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(graph, stream=stream):
-                for i, M in enumerate(MS):
-                    fp6.linear(xs[M], packs[(g * len(MS) + i) % copies], scales, N_DIM, K_DIM,
-                               out=ys[M], workspace=ws)
-            graphs.append(graph)
+        timed_graph = capture(args.steps)
+        warm_graph = capture(args.warmup)
     torch.cuda.synchronize()
 
-    def step(s):
-        graphs[s % n_graphs].replay()
-
     with torch.cuda.stream(stream):
-        for s in range(args.warmup):
-            step(s)
+        warm_graph.replay()
+        timed_graph.replay()                 # first replay of the timed graph itself, untimed
     torch.cuda.synchronize()
     barrier(world)
 
@@ -398,8 +400,7 @@ def run_fp6(args, world, rank, local):
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
         t_start.record()
-        for s in range(args.steps):
-            step(s)
+        timed_graph.replay()                 # exactly args.steps steps
         t_end.record()
     torch.cuda.synchronize()
     barrier(world)
@@ -409,12 +410,9 @@ def run_fp6(args, world, rank, local):
     # this load.
     t_soak = time.perf_counter()
     with torch.cuda.stream(stream):
-        s = 0
         while time.perf_counter() - t_soak < 0.5:
-            step(s)
-            s += 1
-            if s % 64 == 0:
-                stream.synchronize()
+            warm_graph.replay()
+            stream.synchronize()
     torch.cuda.synchronize()
     clocks = sampler.stop(since)
     clocks["window"] = "timed region + 0.5 s of the same graph replays right after it"
@@ -452,20 +450,30 @@ def run_fp6(args, world, rank, local):
             del graph
     per_m = np.array(per_m)
 
-    # end to end through the public API with host buffers: H2D of x, linear, D2H of y
-    x_host = {M: xs[M].cpu().pin_memory() for M in MS}
-    y_host = {M: torch.empty((M, N_DIM), dtype=torch.float16).pin_memory() for M in MS}
-    x_dev = {M: torch.empty_like(xs[M]) for M in MS}
-    h2d = sum(x_host[M].numel() * 2 for M in MS)
-    d2h = sum(y_host[M].numel() * 2 for M in MS)
+    # End to end through the public API with host buffers: every step copies
+    # its five activation matrices host -> device from one pinned staging
+    # buffer, runs the five layer calls (FP6Linear.__call__) and copies their
+    # five outputs device -> host into one pinned buffer.
+    rows = sum(MS)
+    x_host = torch.empty((rows, K_DIM), dtype=torch.float16).pin_memory()
+    y_host = torch.empty((rows, N_DIM), dtype=torch.float16).pin_memory()
+    off = np.cumsum([0] + MS)
+    for M, o in zip(MS, off):
+        x_host[o:o + M].copy_(xs[M].cpu())
+    x_dev = torch.empty((rows, K_DIM), dtype=torch.float16, device=dev)
+    y_dev = torch.empty((rows, N_DIM), dtype=torch.float16, device=dev)
+    x_views = [x_dev[o:o + M] for M, o in zip(MS, off)]
+    y_views = [y_dev[o:o + M] for M, o in zip(MS, off)]
+    layers = [fp6.FP6Linear(p_, scales, N_DIM, K_DIM) for p_ in packs]
+    h2d = x_host.numel() * 2
+    d2h = y_host.numel() * 2
     e2e_steps = max(1, args.steps)
 
     def e2e_step(s):
-        for i, M in enumerate(MS):
-            x_dev[M].copy_(x_host[M], non_blocking=True)
-            fp6.linear(x_dev[M], packs[(s * len(MS) + i) % copies], scales, N_DIM, K_DIM, out=ys[M],
-                       workspace=ws)
-            y_host[M].copy_(ys[M], non_blocking=True)
+        x_dev.copy_(x_host, non_blocking=True)
+        for i in range(len(MS)):
+            layers[(s * len(MS) + i) % copies](x_views[i], out=y_views[i])
+        y_host.copy_(y_dev, non_blocking=True)
 
     with torch.cuda.stream(stream):
         for s in range(args.warmup):

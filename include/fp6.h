@@ -4,9 +4,10 @@
  *
  * The method (FP6-LLM abstract; TC-FPx article, section "kernel solution
  * redesign"): weights are quantized offline to 6-bit floats, pre-packed into
- * aligned 2-bit and 4-bit fragment streams, and at run time a single kernel
- * rebuilds FP16 weights in registers and multiplies them with FP16
- * activations on tensor cores.
+ * aligned 32-bit words (three of every four codes whole in the low six bits
+ * of a byte, the fourth cut into 2-bit pieces kept in the bytes' top bits;
+ * see fp6_prepack), and at run time a single kernel rebuilds FP16 weights in
+ * registers and multiplies them with FP16 activations on tensor cores.
  *
  * Format.  A code is the low 6 bits of a byte: sign (bit 5), exponent e (bits
  * 4..2, bias 3), mantissa m (bits 1..0).  Value: (-1)^s 2^(e-3) (1 + m/4) for
@@ -104,11 +105,11 @@ fp6_status fp6_dequant(const void *packed, const uint16_t *scales, int64_t N, in
                        uint16_t *W16, struct CUstream_st *stream);
 
 /* Bytes of workspace fp6_linear needs for this problem on the current device
- * (0 when the problem is empty).  The first 4096 bytes of a workspace hold
- * counters that must be ZERO before its first use (cudaMemset once); every
- * completed call leaves them zero again, whatever the problem size, so one
- * zeroed buffer of the largest size needed serves every shape.  After a call
- * that reported FP6_ERR_TIMEOUT, zero them again. */
+ * (0 when the problem is empty or unsupported).  The first 16384 bytes of a
+ * workspace hold counters that must be ZERO before its first use (cudaMemset
+ * once); every completed call leaves them zero again, whatever the problem
+ * size, so one zeroed buffer of the largest size needed serves every shape.
+ * After a call that reported FP6_ERR_TIMEOUT, zero them again. */
 size_t fp6_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /*
@@ -161,11 +162,16 @@ fp6_status fp6_selftest_wait_timeout(struct CUstream_st *stream);
  *   Same arguments and result as fp6_linear, without the workspace: the
  *   scratch lives in a fixed 16 MiB array inside the library's device image,
  *   present on every GPU that loads the library until the process exits.
- *   Problems whose fp6_linear_workspace_bytes exceed 16 MiB (on a 148-SM B200,
- *   M > 64) return FP6_ERR_WORKSPACE; use fp6_linear for them.
- *   The first call on each device looks up the array's device address, so make
- *   that first call before capturing a stream.  Each call clears the counters
- *   it needs with cudaMemsetAsync on `stream`; it never allocates or frees.
+ *   A problem whose fp6_linear_workspace_bytes exceed 16 MiB returns
+ *   FP6_ERR_WORKSPACE; use fp6_linear for it.  The workspace grows with the
+ *   token tile and the SM count, not with N or K: on a 148-SM B200 every
+ *   M <= 64 fits and every M > 64 with at least 148 pipeline steps (for
+ *   example any Llama-70B- or OPT-30B-sized layer) does not.
+ *   Each call looks up the array's device address in the current context
+ *   (cudaGetSymbolAddress, which allocates nothing); the first call on a
+ *   device may load the library's device code, so make it before capturing a
+ *   stream.  Each call clears the counters it needs with cudaMemsetAsync on
+ *   `stream`; it never allocates or frees.
  *   All calls on a device share the one array: calls that may overlap on the
  *   GPU (different streams without ordering between them) race and give wrong
  *   results.

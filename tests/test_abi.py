@@ -190,3 +190,8 @@ def test_plan_for_sms_rejects_bad_arguments(lib):
     assert lib.fp6_linear_plan_for_sms(-1, 8192, 8192, 148, out) == 1
     assert lib.fp6_linear_plan_for_sms(1, 100, 8192, 148, out) == 2
     assert lib.fp6_linear_plan_for_sms(1, 8192, 8192, 148, None) == 1
+    # more pipeline steps than the kernels count (2^23 row tiles x 2^26 token
+    # tiles x 2^23 steps would overflow 64-bit step arithmetic): rejected on the
+    # host, before any arithmetic on them
+    assert lib.fp6_linear_plan_for_sms(2 ** 31 - 1, 2 ** 30, 2 ** 30, 148, out) == 2
+    assert lib.fp6_linear_workspace_bytes(2 ** 31 - 1, 2 ** 30, 2 ** 30) == 0

@@ -55,11 +55,23 @@ def _need_cuda(name, t, dtype, dim=None):
         raise ValueError(f"{name} must be contiguous")
 
 
+# Sizes the library reports, cached per shape: a layer called in a decode loop
+# asks for the same few sizes every time, and each query is a foreign call.
+_packed_bytes_cache = {}
+_workspace_cache = {}
+
+
 def packed_bytes(N: int, K: int, fmt=None) -> int:
-    _check_fmt(fmt)
-    if fmt is None:
-        return int(_lib.load().fp6_packed_bytes(N, K))
-    return int(_lib.load().fpx_packed_bytes(fmt, N, K))
+    key = (N, K, fmt)
+    v = _packed_bytes_cache.get(key)
+    if v is None:
+        _check_fmt(fmt)
+        if fmt is None:
+            v = int(_lib.load().fp6_packed_bytes(N, K))
+        else:
+            v = int(_lib.load().fpx_packed_bytes(fmt, N, K))
+        _packed_bytes_cache[key] = v
+    return v
 
 
 def quantize(W, fmt=None):
@@ -116,7 +128,14 @@ def dequant(packed, scales, N: int, K: int, fmt=None):
 
 
 def workspace_bytes(M: int, N: int, K: int) -> int:
-    return int(_lib.load().fp6_linear_workspace_bytes(M, N, K))
+    """Workspace fp6_linear needs on the current device (it depends on the
+    device's SM count, so the cache is keyed by device)."""
+    key = (_torch().cuda.current_device(), M, N, K)
+    v = _workspace_cache.get(key)
+    if v is None:
+        v = int(_lib.load().fp6_linear_workspace_bytes(M, N, K))
+        _workspace_cache[key] = v
+    return v
 
 
 def linear_plan(M: int, N: int, K: int) -> dict:

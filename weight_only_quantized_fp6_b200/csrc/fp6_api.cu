@@ -136,25 +136,33 @@ int stages_for(int ncol) {
   }
 }
 
-bool make_plan(int64_t M, int64_t N, int64_t K, int sms, Plan* pl) {
+// Pipeline steps of one launch at most: the kernels index steps with 64-bit
+// arithmetic (range bounds multiply a step index by the grid size) and count
+// a CTA's own steps in 32 bits.
+constexpr long long kMaxTotalSteps = 1LL << 40;
+
+// The launch plan for an M x N x K problem (shape already checked) on `sms`
+// multiprocessors.  FP6_ERR_UNSUPPORTED_SHAPE when the problem has more
+// pipeline steps than the kernels can count.
+fp6_status make_plan(int64_t M, int64_t N, int64_t K, int sms, Plan* pl) {
   pl->ncol = pick_ncol(M);
   pl->stages = stages_for(pl->ncol);
   pl->n_tiles = static_cast<int>(N / fp6::kTileRows);
   pl->m_tiles = static_cast<int>((M + pl->ncol - 1) / pl->ncol);
   pl->k_tiles = static_cast<int>(K / fp6::kTileCols);
-  pl->tiles = static_cast<long long>(pl->n_tiles) * pl->m_tiles;
+  pl->tiles = static_cast<long long>(pl->n_tiles) * pl->m_tiles;   // < 2^23 * 2^27
   // widest step (power of two up to the variant's limit) that divides K/64
   pl->T = tmax_for(pl->ncol);
   while (pl->T > 1 && pl->k_tiles % pl->T != 0) pl->T >>= 1;
   pl->k_steps = pl->k_tiles / pl->T;
+  if (pl->k_steps > 0 && pl->tiles > kMaxTotalSteps / pl->k_steps) return FP6_ERR_UNSUPPORTED_SHAPE;
   pl->total = pl->tiles * pl->k_steps;
   if (pl->total <= 0) {
     pl->grid = 0;
-    return true;
+    return FP6_OK;
   }
   pl->grid = static_cast<int>(std::min<long long>(std::min(sms, fp6::kMaxGrid), pl->total));
-  // the decode variants (NCOL <= 64) handle one token tile: NCOL >= M
-  if (pl->ncol <= 64 && pl->m_tiles != 1) return false;
+  if ((pl->total + pl->grid - 1) / pl->grid > INT32_MAX) return FP6_ERR_UNSUPPORTED_SHAPE;
   // Many tiles and a nearly full last wave (at most 5 % of the CTA-tile slots
   // idle): whole tiles per CTA, which share weights and activations through
   // L2; otherwise the stream-K ranges balance the work exactly.
@@ -168,7 +176,7 @@ bool make_plan(int64_t M, int64_t N, int64_t K, int sms, Plan* pl) {
   }
   pl->counter_bytes = fp6::kCounterBytes;
   pl->partial_bytes = static_cast<size_t>(2) * pl->grid * pl->ncol * 128 * sizeof(float);
-  return true;
+  return FP6_OK;
 }
 
 // Launches one variant with programmatic dependent launch: the kernel may
@@ -347,7 +355,8 @@ fp6_status linear_impl(const uint16_t* x, const void* packed, const uint16_t* sc
   const int sms = current_device_sms(&dev);
   if (sms <= 0) return FP6_ERR_CUDA;
   Plan pl;
-  make_plan(M, N, K, sms, &pl);
+  st = make_plan(M, N, K, sms, &pl);
+  if (st != FP6_OK) return st;
   const size_t need = pl.counter_bytes + pl.partial_bytes;
   if (workspace_bytes < need || (need > 0 && workspace == nullptr)) return FP6_ERR_WORKSPACE;
   if (need > 0 && !aligned16(workspace)) return FP6_ERR_MISALIGNED;
@@ -445,7 +454,8 @@ fp6_status fp6_linear_plan(int64_t M, int64_t N, int64_t K, int64_t out[5]) {
   const int sms = current_device_sms(&dev);
   if (sms <= 0) return FP6_ERR_CUDA;
   Plan pl;
-  make_plan(M, N, K, sms, &pl);
+  st = make_plan(M, N, K, sms, &pl);
+  if (st != FP6_OK) return st;
   out[0] = pl.ncol;
   out[1] = pl.stages;
   out[2] = pl.grid;
@@ -461,7 +471,8 @@ fp6_status fp6_linear_plan_for_sms(int64_t M, int64_t N, int64_t K, int sms, int
   if (M < 0 || sms <= 0) return FP6_ERR_INVALID_ARG;
   if (M > INT32_MAX) return FP6_ERR_UNSUPPORTED_SHAPE;
   Plan pl;
-  make_plan(M, N, K, sms, &pl);
+  st = make_plan(M, N, K, sms, &pl);
+  if (st != FP6_OK) return st;
   out[0] = pl.ncol;
   out[1] = pl.stages;
   out[2] = pl.grid;
@@ -478,8 +489,7 @@ size_t fp6_linear_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   const int sms = current_device_sms(&dev);
   if (sms <= 0) return 0;
   Plan pl;
-  make_plan(M, N, K, sms, &pl);
-  if (pl.grid == 0) return 0;
+  if (make_plan(M, N, K, sms, &pl) != FP6_OK || pl.grid == 0) return 0;
   return pl.counter_bytes + pl.partial_bytes;
 }
 
@@ -576,22 +586,15 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;   // 16 MiB per device
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
-void* g_noalloc_ptr[kMaxDevices] = {};
-std::mutex g_noalloc_mu;
-
-// Device address of the scratch array on the current device, looked up once
-// per device (the array's host-side name is only a stand-in and must never be
-// handed to a kernel).
+// Device address of the scratch array in the current device's context.  The
+// array's host-side name is only a stand-in and must never be handed to a
+// kernel.  Looked up on every call (it allocates nothing and costs little), so
+// a context that was destroyed and created again, in which the module and
+// its array may sit elsewhere, is never given a stale address.
 fp6_status noalloc_scratch(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FP6_ERR_CUDA;
-  std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) return FP6_ERR_CUDA;
-    g_noalloc_ptr[dev] = ptr;
-  }
-  *out = g_noalloc_ptr[dev];
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) return FP6_ERR_CUDA;
+  *out = ptr;
   return FP6_OK;
 }
 

@@ -46,20 +46,25 @@ __device__ __forceinline__ void cvt_e3m2x4(uint32_t w, uint32_t& o0, uint32_t& o
       : "r"(w));
 }
 
+// The cut codes of one 16-column group (words f0, f1, f2) gathered into the
+// low six bits of four bytes: code bits 5,4 sit in the top bits of f2, bits
+// 3,2 in f1, bits 1,0 in f0.
+__device__ __forceinline__ uint32_t gather_cut(uint32_t f0, uint32_t f1, uint32_t f2) {
+  const uint32_t u1 = (f2 & 0xC0C0C0C0u) | ((f1 >> 2) & 0x3F3F3F3Fu);
+  const uint32_t u2 = (u1 & 0xF0F0F0F0u) | ((f0 >> 4) & 0x0F0F0F0Fu);
+  return u2 >> 2;
+}
+
 // Rebuild the 64 fp16 weights (as 32 fp16x2 words, low half = even column)
 // of one row of one tile from its 12 words: decode(c) exactly.
 __device__ __forceinline__ void splice_row(const uint32_t (&F)[kRowWords], uint32_t (&out)[32]) {
 #pragma unroll
   for (int g = 0; g < 4; ++g) {
     const uint32_t f0 = F[3 * g], f1 = F[3 * g + 1], f2 = F[3 * g + 2];
-    // cut codes: top bits of f2 (code bits 5,4), f1 (3,2), f0 (1,0) -> bits 5..0
-    const uint32_t u1 = (f2 & 0xC0C0C0C0u) | ((f1 >> 2) & 0x3F3F3F3Fu);
-    const uint32_t u2 = (u1 & 0xF0F0F0F0u) | ((f0 >> 4) & 0x0F0F0F0Fu);
-    const uint32_t t = u2 >> 2;
     cvt_e3m2x4(f0, out[8 * g + 0], out[8 * g + 1]);
     cvt_e3m2x4(f1, out[8 * g + 2], out[8 * g + 3]);
     cvt_e3m2x4(f2, out[8 * g + 4], out[8 * g + 5]);
-    cvt_e3m2x4(t, out[8 * g + 6], out[8 * g + 7]);
+    cvt_e3m2x4(gather_cut(f0, f1, f2), out[8 * g + 6], out[8 * g + 7]);
   }
 }
 
@@ -204,15 +209,13 @@ struct Format<Fmt::E2M3> {
 #pragma unroll
     for (int g = 0; g < 4; ++g) {
       const uint32_t f0 = F[3 * g], f1 = F[3 * g + 1], f2 = F[3 * g + 2];
-      const uint32_t u1 = (f2 & 0xC0C0C0C0u) | ((f1 >> 2) & 0x3F3F3F3Fu);
-      const uint32_t u2 = (u1 & 0xF0F0F0F0u) | ((f0 >> 4) & 0x0F0F0F0Fu);
-      const uint32_t t = u2 >> 2;
       cvt_e2m3x4(f0, out[8 * g + 0], out[8 * g + 1]);
       cvt_e2m3x4(f1, out[8 * g + 2], out[8 * g + 3]);
       cvt_e2m3x4(f2, out[8 * g + 4], out[8 * g + 5]);
-      cvt_e2m3x4(t, out[8 * g + 6], out[8 * g + 7]);
+      cvt_e2m3x4(gather_cut(f0, f1, f2), out[8 * g + 6], out[8 * g + 7]);
     }
   }
+
   __device__ static void pack(const uint8_t (&c)[64], uint32_t (&F)[kRowWords]) { pack_row(c, F); }
   __device__ static void store(uint8_t* tile, int r, const uint32_t (&F)[kRowWords]) { store_row_words(tile, r, F); }
 };
@@ -245,6 +248,7 @@ struct Format<Fmt::E2M1> {
       for (int b = 0; b < 4; ++b) out[4 * w + b] = o[b];
     }
   }
+
   __device__ static void pack(const uint8_t (&c)[64], uint32_t (&F)[kRowWords]) {
 #pragma unroll
     for (int w = 0; w < kRowWords; ++w) F[w] = 0;
@@ -291,6 +295,7 @@ struct Format<Fmt::E2M2> {
       }
     }
   }
+
   __device__ static void pack(const uint8_t (&c)[64], uint32_t (&F)[kRowWords]) {
 #pragma unroll
     for (int w = 0; w < kRowWords; ++w) F[w] = 0;

@@ -71,7 +71,7 @@ constexpr int kWProdWarp = kFirstDeqWarp + 4 * kDeqGroups;   // 20
 constexpr int kXProdWarp = kWProdWarp + 1;                   // 21
 constexpr int kLinearThreads = 32 * (kXProdWarp + 1);        // 704
 constexpr int kMaxGrid = 1024;                // persistent CTAs at most (one per SM)
-constexpr int kCounterBytes = kMaxGrid * 4;
+constexpr int kCounterBytes = kMaxGrid * 16;   // up to four counters per CTA
 constexpr uint32_t kTmemCols = 512;
 
 template <int NCOL, Fmt F = Fmt::E3M2>
@@ -139,6 +139,7 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
   const bool ok = wait_bounded(bar, parity, abort);
   return __all_sync(0xffffffffu, ok) != 0;
 }
+
 
 // Walks the CTA's steps: the step index within the tile and the tile's (row
 // tile, token tile) coordinates, advanced without divisions.

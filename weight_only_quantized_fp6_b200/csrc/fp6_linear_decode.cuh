@@ -3,11 +3,10 @@
 //
 // Same product and the same work split as fp6_linear_kernel (fp6_linear.cuh):
 // y[M,N] = x[M,K] . (scale (.) decode(W[N,K]))^T, fp32 accumulation, fp16 out,
-// persistent CTAs over equal ranges of (row tile, step) iterations, split
-// tiles finished, in CTA order, by the CTA holding their first steps.  What differs is the
-// pipeline, shaped for the memory-bound regime where the tensor core is nearly
-// idle and the integer pipe (the FP6 -> FP16 splice) and synchronisation
-// latency are what remain:
+// persistent CTAs over equal ranges of (row tile, step) iterations.  What
+// differs is the pipeline, shaped for the memory-bound regime where the
+// tensor core is nearly idle and the integer pipe (the FP6 -> FP16 splice)
+// and synchronisation latency are what remain:
 //
 //   warps 0..4G-1 G dequant groups of four warps (one per TMEM lane
 //                 quadrant), taking every G-th step (G = 3; G = 2 for 64 token
@@ -40,6 +39,20 @@
 // Ring ownership keeps every mbarrier's waits in phase order: weight stages
 // (SW) are a multiple of G and x stages are the TMEM slots, so each stage is
 // always used by the same group; slots and accumulators belong to one group.
+//
+// Split row tiles.  A row tile whose steps span CTAs c_lo .. c_hi is finished
+// by exactly one of them, and no CTA ever waits for another (so nothing
+// depends on the CTAs of a launch being resident at the same time).  Each
+// epilogue warp (32 rows) has its own counter per tile.  Every contributor
+// after c_lo reaches the tile at the start of its range, writes its partial
+// sums and adds one to the counter (release).  c_lo reaches the tile at the
+// end of its range; if the counter shows every other contributor (acquire),
+// it sums their partials with its own accumulators and stores y.  Otherwise
+// it writes its own partial and adds one as well, and whichever contributor's
+// add completes the count sums the partials.  The sum is always formed in the
+// same order (contributors c_lo+1 .. c_hi, then c_lo), so results are
+// bit-reproducible whichever CTA finishes the tile.  The finisher resets the
+// counter to zero for the next launch.
 //
 // The role loops never leave early: a warp whose bounded wait gave up (the
 // abort flag is raised) skips its work but still makes every later arrival,
@@ -91,8 +104,8 @@ struct DecodeShape {
   static constexpr int kWOff = kRX * kXStage;
   static constexpr int kBarOff = kWOff + kSW * kWStage;
   // wfull, wempty [SW]; xfull [RX]; slot free [slots] (frees the x stage too);
-  // slot ready [slots]; dfull, dempty [2]; epi [2]; done
-  static constexpr int kNumBars = 2 * kSW + kRX + 2 * kSlots + 2 + 2 + 2 + 1;
+  // slot ready [slots]; dfull, dempty [2]; done
+  static constexpr int kNumBars = 2 * kSW + kRX + 2 * kSlots + 2 + 2 + 1;
   static constexpr int kBarrierBytes = 1024;
   static constexpr int kSmemBytes = kBarOff + kBarrierBytes + 1024;  // + alignment slack
   static_assert(kSW % kGroups == 0 && kRX == kSlots, "stages owned by one group; one x stage per slot");
@@ -116,6 +129,13 @@ __device__ __forceinline__ int group_first(int g, int a, int groups) {
   return a + ((g - a % groups) + groups) % groups;
 }
 
+// Partial sums of a split tile, [2G][NCOL][128] fp32: slot 2c for the tile a
+// CTA's range starts in, 2c + 1 for the one it ends in.
+template <int NCOL>
+__device__ __forceinline__ float* decode_partial(float* partials, int slot, int r) {
+  return partials + static_cast<long long>(slot) * NCOL * 128 + r;
+}
+
 template <int NCOL, Fmt F = Fmt::E3M2>
 __global__ void __launch_bounds__(DecodeShape<NCOL, F>::kThreads, 1)
     fp6_linear_decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const LinearParams p) {
@@ -133,11 +153,9 @@ __global__ void __launch_bounds__(DecodeShape<NCOL, F>::kThreads, 1)
   uint64_t* slotready = slotfree + S::kSlots;     // [slots]: the group's four warps have written the slot
   uint64_t* dfull = slotready + S::kSlots;        // [2]: a segment's accumulators are complete
   uint64_t* dempty = dfull + 2;                   // [2]: the epilogue has read them
-  uint64_t* epi = dempty + 2;                     // [2]: fix-up meeting (epi[0] only)
-  uint64_t* done = epi + 2;                       // every MMA finished (before TMEM release)
+  uint64_t* done = dempty + 2;                    // every MMA finished (before TMEM release)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + S::kNumBars);
-  volatile int* s_last = reinterpret_cast<volatile int*>(tmem_holder + 1);  // [2]
-  volatile int* s_abort = s_last + 2;
+  volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_holder + 1);
   volatile int* s_never = s_abort + 1;
 
   const int warp = threadIdx.x >> 5;
@@ -165,14 +183,12 @@ __global__ void __launch_bounds__(DecodeShape<NCOL, F>::kThreads, 1)
     else if (b >= bs && b < br) count = S::kIss;              // slotfree: the group's issuers
     else if (b >= br && b < bd) count = 4;                    // slotready: the group's four warps
     else if (b >= bd && b < bd + 2) count = S::kGroups * S::kIss;  // dfull: one arrival per issuer
-    else if (b >= bd + 2 && b < bd + 6) count = 4;            // dempty, epi: epilogue warps
-    else if (b == bd + 6) count = S::kGroups * S::kIss;       // done: one commit per issuer
+    else if (b >= bd + 2 && b < bd + 4) count = 4;            // dempty: epilogue warps
+    else if (b == bd + 4) count = S::kGroups * S::kIss;       // done: one commit per issuer
     mbar_init(smem_u32(&bars[b]), count);
     fence_barrier_init();
   }
   if (threadIdx.x == 0) {
-    s_last[0] = 0;
-    s_last[1] = 0;
     *s_abort = 0;
     *s_never = 0;
   }
@@ -328,14 +344,7 @@ __global__ void __launch_bounds__(DecodeShape<NCOL, F>::kThreads, 1)
     warp_wait(smem_u32(done), 0, s_never);
   } else if (warp >= S::kEpiWarp && warp < S::kEpiWarp + 4) {
     // ---------------- epilogue warpgroup: segments in order ----------------
-    // A split row tile is finished by its first CTA c_lo, which reaches the
-    // tile at the end of its range; every later contributor reaches it at the
-    // start of its own range, publishes its partial there (release add on the
-    // tile's counter) and moves on.  The finishing CTA waits for those
-    // partials and sums them (in CTA order) while its own MMAs still run, so
-    // the end of its range costs one TMEM read and the store of y.  Each
-    // epilogue warp of a contributor releases its 32 rows with one add, so the
-    // counter reaches 4 per contributor.
+    // Split row tiles: see the fix-up protocol at the top of this file.
     grid_dependency_wait();                  // y, partials and counters may be in use before this kernel
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
@@ -344,6 +353,7 @@ __global__ void __launch_bounds__(DecodeShape<NCOL, F>::kThreads, 1)
     for (int sg = 0; sg < nseg; ++sg) {
       const long long tile = tile_first + sg;
       const int set = sg % S::kSets;
+      const uint32_t dpar = (sg / S::kSets) & 1;
       int a, b;
       segment_range(sg, tile_first, s0, KS, n_local, &a, &b);
       const int n = static_cast<int>(tile) * kTileRows + r;
@@ -352,35 +362,15 @@ __global__ void __launch_bounds__(DecodeShape<NCOL, F>::kThreads, 1)
       const int c_hi = range_owner(tile * KS + KS - 1, total, G);
       const bool split = c_lo != c_hi;
       const bool finisher = (c == c_lo);
-      float pre[NCOL];
-#pragma unroll
-      for (int j = 0; j < NCOL; ++j) pre[j] = 0.0f;
-      if (split && finisher) {
-        // the other contributors' partials, summed in CTA order
-        if (!wait_counter(&p.counters[c_lo], 4u * static_cast<unsigned int>(c_hi - c_lo), s_abort)) break;
-        for (int cc = c_lo + 1; cc <= c_hi; ++cc) {
-          const float* src = p.partials + static_cast<long long>(cc) * NCOL * 128 + r;
-#pragma unroll
-          for (int j = 0; j < NCOL; ++j)
-            if (j < mcount) pre[j] += __ldcg(src + j * 128);
-        }
-        // Reset the counter for the next launch once all four warps have seen
-        // it complete (a CTA finishes at most one split tile: one meeting).
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&epi[0]));
-        if (quad == 0 && warp_wait(smem_u32(&epi[0]), 0, s_abort) && lane == 0) p.counters[c_lo] = 0u;
-      }
-      if (!warp_wait(smem_u32(&dfull[set]), (sg / S::kSets) & 1, s_abort)) break;
-      tc_fence_after();
-      float* part = p.partials + static_cast<long long>(c) * NCOL * 128 + r;
-#pragma unroll
-      for (int ch = 0; ch < NCOL / 8; ++ch) {
-        const int c0 = ch * 8;
-        if (c0 >= mcount) break;
-        float acc[8];
+      const unsigned int need = static_cast<unsigned int>(c_hi - c_lo);   // adds of the later contributors
+      unsigned int* cnt = p.counters + 4 * c_lo + quad;
+      uint16_t* ybase = p.y + n;
+
+      // This segment's own sums, columns c0 .. c0+7: the accumulators of the
+      // groups (and their issuers) added in a fixed order.
+      auto own8 = [&](int c0, float (&acc)[8]) {
 #pragma unroll
         for (int jj = 0; jj < 8; ++jj) acc[jj] = 0.0f;
-        // groups in order: the sum is the same on every run
         for (int g = 0; g < S::kGroups; ++g) {
           if (group_first(g, a, S::kGroups) > b) continue;   // no step of group g in this segment
           for (int i = 0; i < S::kIss; ++i) {
@@ -391,25 +381,144 @@ __global__ void __launch_bounds__(DecodeShape<NCOL, F>::kThreads, 1)
             for (int jj = 0; jj < 8; ++jj) acc[jj] += __uint_as_float(v[jj]);
           }
         }
-        if (split && !finisher) {
+      };
+      // Partials of contributors c_lo+1 .. c_hi summed in CTA order, columns
+      // c0 .. c0+7.
+      auto others8 = [&](int c0, float (&q)[8]) {
 #pragma unroll
-          for (int jj = 0; jj < 8; ++jj) __stcg(part + (c0 + jj) * 128, acc[jj]);
-        } else {
+        for (int jj = 0; jj < 8; ++jj) q[jj] = 0.0f;
+        for (int cc = c_lo + 1; cc <= c_hi; ++cc) {
+          const float* src = decode_partial<NCOL>(p.partials, 2 * cc, r) + c0 * 128;
 #pragma unroll
-          for (int jj = 0; jj < 8; ++jj) {
-            const float v = pre[c0 + jj] + acc[jj];
-            if (c0 + jj < mcount)
-              p.y[static_cast<long long>(c0 + jj) * p.N + n] = __half_as_ushort(__float2half_rn(v * mul));
+          for (int jj = 0; jj < 8; ++jj) q[jj] += __ldcg(src + jj * 128);
+        }
+      };
+      auto store8 = [&](int c0, const float (&v)[8]) {
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj)
+          if (c0 + jj < mcount)
+            ybase[static_cast<long long>(c0 + jj) * p.N] = __half_as_ushort(__float2half_rn(v[jj] * mul));
+      };
+      // The accumulators of this set are read: the issuers may reuse them.
+      auto release = [&]() {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&dempty[set]));
+      };
+      // Write this CTA's partial (slot 2c + which), release the accumulators
+      // and add one to the counter; true when this add completed the count
+      // (every other contributor, c_lo included, had counted), making this
+      // warp the one that finishes the tile, from the partials in memory.
+      auto publish = [&](int which) -> bool {
+        float* mine = decode_partial<NCOL>(p.partials, 2 * c + which, r);
+#pragma unroll
+        for (int c0 = 0; c0 < NCOL; c0 += 8) {
+          if (c0 >= mcount) break;
+          float acc[8];
+          own8(c0, acc);
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) __stcg(mine + (c0 + jj) * 128, acc[jj]);
+        }
+        // The lanes' partial stores are ordered before lane 0's add by the
+        // warp barrier, and its release publishes them with its own.
+        release();
+        unsigned int old = 0;
+        if (lane == 0) old = atom_add_acq_rel(cnt, 1u);
+        const bool last = __shfl_sync(0xffffffffu, old, 0) == need;
+        if (last) (void)ld_acquire(cnt);      // every lane acquires the others' partials
+        return last;
+      };
+      // The whole tile from the partials in memory: contributors c_lo+1 ..
+      // c_hi in CTA order, then c_lo's.
+      auto finish_from_partials = [&]() {
+        const float* lo = decode_partial<NCOL>(p.partials, 2 * c_lo + 1, r);
+#pragma unroll
+        for (int c0 = 0; c0 < NCOL; c0 += 8) {
+          if (c0 >= mcount) break;
+          float q[8];
+          others8(c0, q);
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) q[jj] += __ldcg(lo + (c0 + jj) * 128);
+          store8(c0, q);
+        }
+        __syncwarp();
+        if (lane == 0) *cnt = 0u;            // every contributor has counted: reset for the next launch
+      };
+      // Every later contributor has counted (each lane acquires on its own).
+      auto all_counted = [&]() -> bool {
+        return __all_sync(0xffffffffu, ld_acquire(cnt) == need) != 0;
+      };
+
+      if (!split) {
+        if (!warp_wait(smem_u32(&dfull[set]), dpar, s_abort)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int c0 = 0; c0 < NCOL; c0 += 8) {
+          if (c0 >= mcount) break;
+          float acc[8];
+          own8(c0, acc);
+          store8(c0, acc);
+        }
+        release();
+      } else if (finisher) {
+        // With 16 token columns the others' partials fit in registers: sum
+        // them while this CTA's last MMAs still run, as soon as all are there.
+        float pre[16];
+        bool pre_ok = false;
+        if constexpr (NCOL == 16) {
+          while (true) {
+            if (all_counted()) {
+#pragma unroll
+              for (int c0 = 0; c0 < 16; c0 += 8) {
+                float q[8];
+                others8(c0, q);
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) pre[c0 + jj] = q[jj];
+              }
+              pre_ok = true;
+              break;
+            }
+            const bool fin = mbar_try_wait(smem_u32(&dfull[set]), dpar);
+            if (__any_sync(0xffffffffu, fin || *s_abort)) break;
+            __nanosleep(128);
           }
         }
-      }
-      // accumulators read: the set may be reused kSets segments on
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&dempty[set]));
-      if (split && !finisher) {
-        __syncwarp();                        // the warp's partial rows are written
-        if (lane == 0) red_release_add(&p.counters[c_lo], 1u);
+        if (!warp_wait(smem_u32(&dfull[set]), dpar, s_abort)) break;
+        tc_fence_after();
+        if (pre_ok || all_counted()) {
+#pragma unroll
+          for (int c0 = 0; c0 < NCOL; c0 += 8) {
+            if (c0 >= mcount) break;
+            float acc[8], q[8];
+            own8(c0, acc);
+            if constexpr (NCOL == 16) {
+              if (pre_ok) {
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) q[jj] = pre[(c0 + jj) & 15];
+              } else {
+                others8(c0, q);
+              }
+            } else {
+              others8(c0, q);
+            }
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) acc[jj] = q[jj] + acc[jj];
+            store8(c0, acc);
+          }
+          release();
+          __syncwarp();
+          if (lane == 0) *cnt = 0u;          // every contributor has counted: reset for the next launch
+        } else if (publish(1)) {
+          // Not every partial was there; they all are now, after this one.
+          finish_from_partials();
+        }
+      } else {
+        // A later contributor (this tile is where its range starts).
+        if (!warp_wait(smem_u32(&dfull[set]), dpar, s_abort)) break;
+        tc_fence_after();
+        // If c_lo and every other contributor counted before this one, this
+        // warp finishes the tile, in the order c_lo would.
+        if (publish(0)) finish_from_partials();
       }
     }
   }

@@ -87,35 +87,19 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, vola
 }
 
 // ---- cross-CTA counters in global memory ---------------------------------------
-// Add to a counter with release semantics at GPU scope: every earlier write
-// of this thread is visible to a thread that reads the new value with acquire.
-__device__ __forceinline__ void red_release_add(unsigned int* p, unsigned int v) {
-  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
 __device__ __forceinline__ unsigned int ld_acquire(const unsigned int* p) {
   unsigned int v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
-// Wait until *p == target (another CTA's releases).  Gives up after
-// kWaitLimitNs or once *abort is raised, like wait_bounded().
-__device__ __forceinline__ bool wait_counter(const unsigned int* p, unsigned int target, volatile int* abort) {
-  if (ld_acquire(p) == target) return true;
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t i = 1;; ++i) {
-    __nanosleep(64);
-    if (ld_acquire(p) == target) return true;
-    if ((i & 3u) == 0) {
-      if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        *abort = 1;
-        atomicOr(&g_error_word, kErrTimeout);
-        return false;
-      }
-    }
-  }
+// Add to a counter with acquire-release semantics at GPU scope and return the
+// previous value: the adding thread's earlier writes are published, and the
+// writes published by earlier adders become visible to it.
+__device__ __forceinline__ unsigned int atom_add_acq_rel(unsigned int* p, unsigned int v) {
+  unsigned int old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
 }
-
 // ---- bulk copies (no multicast anywhere in this library) ---------------------
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar,
                                           uint64_t policy) {
