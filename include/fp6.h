@@ -241,6 +241,55 @@ fp6_status fpx_linear(fpx_format fmt, const uint16_t *x, const void *packed, con
                       int64_t M, int64_t N, int64_t K, uint16_t *y,
                       void *workspace, size_t workspace_bytes, struct CUstream_st *stream);
 
+/*
+ * 2:4 structured-sparse INT4 weights (NEXT-4; the Sparse-Marlin post: 4-bit
+ * weights with 2:4 sparsity, metadata giving the kept positions, per-row
+ * quantization statistics).  The post fixes none of the details; these
+ * entry points take the plain readings:
+ *   pruning  in each group of 4 consecutive weights of a row (k = 4j..4j+3)
+ *            the two with the largest |w| are kept, ties to the lower position;
+ *   scale    scale[n] = fp16_rne( fp32( max_k |W[n,k]| / 7 ) );
+ *   codes    q = round-half-even(w / scale) clamped to [-8, 7];
+ *   value    scale * q at the kept positions, 0 elsewhere.
+ * Same conventions, status codes, workspace (fp6_linear_workspace_bytes) and
+ * launch rules as the fp6_* functions.  The layer runs through the same fused
+ * kernels, whose rebuild expands each group's two codes to four fp16 values.
+ */
+
+/* 3*N*K/8 bytes (two 4-bit codes and two 2-bit positions per four weights);
+ * 0 for unsupported shapes. */
+size_t s24_packed_bytes(int64_t N, int64_t K);
+
+/* W [N,K] fp32 (K % 4 == 0, else FP6_ERR_UNSUPPORTED_SHAPE) ->
+ *   q      [N,K/2] int8, device: the two kept codes of each group, in position order
+ *   pos    [N,K/2] uint8, device: their positions 0..3 within the group (pos[2j] < pos[2j+1])
+ *   scales [N] fp16 bit patterns, device
+ * SYNCHRONIZES the stream to report FP6_ERR_NONFINITE or FP6_ERR_SCALE_RANGE,
+ * as fp6_quantize.  A row of zeros gets scale 0, codes 0 and positions 0, 1. */
+fp6_status s24_quantize(const float *W, int64_t N, int64_t K, int8_t *q, uint8_t *pos,
+                        uint16_t *scales, struct CUstream_st *stream);
+
+/* q, pos as produced by s24_quantize -> packed, s24_packed_bytes(N,K) bytes:
+ *   tiles of 128 rows x 64 columns, tile (nt, kt) at byte (nt*(K/64)+kt)*3072;
+ *   row r of a tile owns four code words V_w at byte r*16 + 4w and two
+ *   position words P_h at byte 2048 + r*8 + 4h.  Group j (0..15) of the tile
+ *   row keeps its codes in byte j%4 of V_{j/4} (first code in the low nibble,
+ *   4-bit two's complement) and its positions in bits 4(j%8)..4(j%8)+3 of
+ *   P_{j/8} (i0 in the low two bits, i1 in the next two).  Little-endian. */
+fp6_status s24_prepack(const int8_t *q, const uint8_t *pos, int64_t N, int64_t K,
+                       void *packed, size_t packed_bytes, struct CUstream_st *stream);
+
+/* Dense fp16 weights: fp16(q) at the kept positions without scales,
+ * fp16_rne(scale * q) with them; +0 at the pruned positions. */
+fp6_status s24_dequant(const void *packed, const uint16_t *scales, int64_t N, int64_t K,
+                       uint16_t *W16, struct CUstream_st *stream);
+
+/* y[M,N] = x[M,K] . (scale (.) v)^T with v the dense code values, fp32
+ * accumulation, fp16 output; arguments and workspace as fp6_linear. */
+fp6_status s24_linear(const uint16_t *x, const void *packed, const uint16_t *scales,
+                      int64_t M, int64_t N, int64_t K, uint16_t *y,
+                      void *workspace, size_t workspace_bytes, struct CUstream_st *stream);
+
 #ifdef __cplusplus
 }
 #endif

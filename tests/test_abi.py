@@ -19,7 +19,7 @@ def lib():
 def declared_functions():
     src = open(os.path.join(ROOT, "include", "fp6.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(fp[6x]_[a-z_0-9]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b((?:fp[6x]|s24)_[a-z_0-9]+)\s*\(", src)))
 
 
 def test_every_declared_symbol_is_exported(lib):
@@ -39,7 +39,7 @@ def declared_arities():
     src = open(os.path.join(ROOT, "include", "fp6.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     out = {}
-    for m in re.finditer(r"\b(fp[6x]_[a-z_0-9]+)\s*\(([^)]*)\)\s*;", src):
+    for m in re.finditer(r"\b((?:fp[6x]|s24)_[a-z_0-9]+)\s*\(([^)]*)\)\s*;", src):
         params = m.group(2).strip()
         out[m.group(1)] = 0 if params in ("", "void") else len(params.split(","))
     return out

@@ -10,7 +10,9 @@ the library's CUDA kernels.
 
 Every function takes an optional `fmt`: None (the default) is FP6 e3m2 through
 the fp6_* entry points; E3M2, E2M3 (FP6 with two exponent bits), E2M1 (FP4)
-or E2M2 (FP5) select the fpx_* entry points with that format.
+or E2M2 (FP5) select the fpx_* entry points with that format, and S24 the
+2:4-sparse INT4 weights of the s24_* entry points (quantized by
+s24_quantize, which also returns the kept positions).
 """
 from __future__ import annotations
 
@@ -21,16 +23,17 @@ from . import _lib
 
 __all__ = ["quantize", "prepack", "dequant", "linear", "linear_plan", "workspace_bytes",
            "packed_bytes", "device_status", "FP6Linear", "FP6Error", "Workspace",
-           "E3M2", "E2M3", "E2M1", "E2M2"]
+           "s24_quantize", "s24_prepack", "E3M2", "E2M3", "E2M1", "E2M2", "S24"]
 
 FP6Error = _lib.FP6Error
 
-# fpx_format values (include/fp6.h)
+# fpx_format values (include/fp6.h); S24 selects the s24_* entry points
 E3M2, E2M3, E2M1, E2M2 = 0, 1, 2, 3
+S24 = 4
 
 
 def _check_fmt(fmt):
-    if fmt is not None and fmt not in (E3M2, E2M3, E2M1, E2M2):
+    if fmt is not None and fmt not in (E3M2, E2M3, E2M1, E2M2, S24):
         raise ValueError(f"unknown format {fmt!r}")
 
 
@@ -68,6 +71,8 @@ def packed_bytes(N: int, K: int, fmt=None) -> int:
         _check_fmt(fmt)
         if fmt is None:
             v = int(_lib.load().fp6_packed_bytes(N, K))
+        elif fmt == S24:
+            v = int(_lib.load().s24_packed_bytes(N, K))
         else:
             v = int(_lib.load().fpx_packed_bytes(fmt, N, K))
         _packed_bytes_cache[key] = v
@@ -78,6 +83,8 @@ def quantize(W, fmt=None):
     """W [N,K] fp32 (cuda) -> (codes [N,K] uint8, scales [N] fp16).  Synchronizes."""
     torch = _torch()
     _check_fmt(fmt)
+    if fmt == S24:
+        raise ValueError("2:4 sparse weights are quantized by s24_quantize")
     _need_cuda("W", W, torch.float32, 2)
     N, K = W.shape
     codes = torch.empty((N, K), dtype=torch.uint8, device=W.device)
@@ -94,6 +101,8 @@ def quantize(W, fmt=None):
 def prepack(codes, fmt=None):
     """codes [N,K] uint8 (cuda) -> packed uint8 buffer (3*N*K/4 bytes; N*K/2 for E2M1, 5*N*K/8 for E2M2)."""
     torch = _torch()
+    if fmt == S24:
+        raise ValueError("2:4 sparse weights are packed by s24_prepack")
     _need_cuda("codes", codes, torch.uint8, 2)
     N, K = codes.shape
     nbytes = packed_bytes(N, K, fmt)
@@ -121,10 +130,43 @@ def dequant(packed, scales, N: int, K: int, fmt=None):
     lib = _lib.load()
     if fmt is None:
         st = lib.fp6_dequant(packed.data_ptr(), sp, N, K, out.data_ptr(), _stream(packed))
+    elif fmt == S24:
+        st = lib.s24_dequant(packed.data_ptr(), sp, N, K, out.data_ptr(), _stream(packed))
     else:
         st = lib.fpx_dequant(fmt, packed.data_ptr(), sp, N, K, out.data_ptr(), _stream(packed))
     _lib.check(st, "fp6_dequant" if fmt is None else "fpx_dequant")
     return out
+
+
+def s24_quantize(W):
+    """W [N,K] fp32 (cuda, K % 4 == 0) -> (q [N,K/2] int8, pos [N,K/2] uint8,
+    scales [N] fp16): in each group of four the two largest |w| kept, their
+    codes round-half-even(w/scale) in [-8, 7] and positions.  Synchronizes."""
+    torch = _torch()
+    _need_cuda("W", W, torch.float32, 2)
+    N, K = W.shape
+    q = torch.empty((N, K // 2), dtype=torch.int8, device=W.device)
+    pos = torch.empty((N, K // 2), dtype=torch.uint8, device=W.device)
+    scales = torch.empty((N,), dtype=torch.float16, device=W.device)
+    st = _lib.load().s24_quantize(W.data_ptr(), N, K, q.data_ptr(), pos.data_ptr(), scales.data_ptr(), _stream(W))
+    _lib.check(st, "s24_quantize")
+    return q, pos, scales
+
+
+def s24_prepack(q, pos):
+    """(q, pos) [N,K/2] -> packed uint8 buffer of 3*N*K/8 bytes."""
+    torch = _torch()
+    _need_cuda("q", q, torch.int8, 2)
+    _need_cuda("pos", pos, torch.uint8, 2)
+    N, K2 = q.shape
+    K = 2 * K2
+    nbytes = packed_bytes(N, K, S24)
+    if nbytes == 0 and N * K > 0:
+        raise FP6Error(2, "s24_prepack")
+    packed = torch.empty((nbytes,), dtype=torch.uint8, device=q.device)
+    st = _lib.load().s24_prepack(q.data_ptr(), pos.data_ptr(), N, K, packed.data_ptr(), nbytes, _stream(q))
+    _lib.check(st, "s24_prepack")
+    return packed
 
 
 def workspace_bytes(M: int, N: int, K: int) -> int:
@@ -197,6 +239,8 @@ def linear(x, packed, scales, N: int, K: int, out=None, workspace: Workspace | N
     lib = _lib.load()
     if fmt is None:
         _lib.check(lib.fp6_linear(*args), "fp6_linear")
+    elif fmt == S24:
+        _lib.check(lib.s24_linear(*args), "s24_linear")
     else:
         _lib.check(lib.fpx_linear(fmt, *args), "fpx_linear")
     return out
@@ -220,6 +264,9 @@ class FP6Linear:
 
     @classmethod
     def from_float(cls, W, fmt=None):
+        if fmt == S24:
+            q, pos, scales = s24_quantize(W)
+            return cls(s24_prepack(q, pos), scales, W.shape[0], W.shape[1], fmt)
         codes, scales = quantize(W, fmt)
         return cls(prepack(codes, fmt), scales, W.shape[0], W.shape[1], fmt)
 

@@ -42,6 +42,11 @@ SIGNATURES = {
     "fpx_prepack": (_ST, [_ST, _P, _I64, _I64, _P, _SZ, _P]),
     "fpx_dequant": (_ST, [_ST, _P, _P, _I64, _I64, _P, _P]),
     "fpx_linear": (_ST, [_ST, _P, _P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
+    "s24_packed_bytes": (_SZ, [_I64, _I64]),
+    "s24_quantize": (_ST, [_P, _I64, _I64, _P, _P, _P, _P]),
+    "s24_prepack": (_ST, [_P, _P, _I64, _I64, _P, _SZ, _P]),
+    "s24_dequant": (_ST, [_P, _P, _I64, _I64, _P, _P]),
+    "s24_linear": (_ST, [_P, _P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
 }
 
 _lock = threading.Lock()

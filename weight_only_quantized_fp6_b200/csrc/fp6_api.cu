@@ -54,7 +54,7 @@ fp6_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FP6_OK : FP6_E
 // ---- per-device cached properties ------------------------------------------
 struct DeviceInfo {
   int sms = 0;
-  bool attrs_set[4][10] = {};  // [format][kernel variant]: shared-memory limit raised
+  bool attrs_set[5][10] = {};  // [format][kernel variant]: shared-memory limit raised
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -272,6 +272,7 @@ size_t packed_bytes_of(Fmt f, int64_t N, int64_t K) {
   switch (f) {
     case Fmt::E2M1: return nk / 2;
     case Fmt::E2M2: return nk / 8 * 5;
+    case Fmt::S24: return nk / 8 * 3;
     default: return nk / 4 * 3;
   }
 }
@@ -329,9 +330,9 @@ fp6_status dequant_impl(const void* packed, const uint16_t* scales, int64_t N, i
   if (N == 0 || K == 0) return FP6_OK;
   if (!packed || !W16) return FP6_ERR_INVALID_ARG;
   if (!aligned16(packed) || !aligned16(W16) || (scales && !aligned16(scales))) return FP6_ERR_MISALIGNED;
-  const int64_t work = N * (K / fp6::kTileCols);
-  const int64_t blocks = (work + 255) / 256;
-  fp6::dequant_kernel<F><<<static_cast<unsigned int>(blocks), 256, 0, stream>>>(
+  const int64_t units = (N / 32) * (K / fp6::kTileCols);   // 32 rows of one tile per warp
+  const int64_t blocks = std::min<int64_t>((units + fp6::kDequantWarps - 1) / fp6::kDequantWarps, 1 << 20);
+  fp6::dequant_kernel<F><<<static_cast<unsigned int>(blocks), 32 * fp6::kDequantWarps, 0, stream>>>(
       static_cast<const uint8_t*>(packed), scales, N, K, W16);
   return cuda_status(cudaGetLastError());
 }
@@ -552,6 +553,60 @@ fp6_status fpx_linear(fpx_format fmt, const uint16_t* x, const void* packed, con
     case Fmt::E2M1: return linear_impl<Fmt::E2M1>(x, packed, scales, M, N, K, y, workspace, workspace_bytes, stream);
     default: return linear_impl<Fmt::E2M2>(x, packed, scales, M, N, K, y, workspace, workspace_bytes, stream);
   }
+}
+
+// ---- 2:4 sparse INT4 (Sparse-Marlin) ------------------------------------------
+size_t s24_packed_bytes(int64_t N, int64_t K) {
+  if (check_shape(N, K) != FP6_OK) return 0;
+  return packed_bytes_of(Fmt::S24, N, K);
+}
+
+fp6_status s24_quantize(const float* W, int64_t N, int64_t K, int8_t* q, uint8_t* pos, uint16_t* scales,
+                        cudaStream_t stream) {
+  if (N < 0 || K < 0) return FP6_ERR_INVALID_ARG;
+  if (K % 4 != 0) return FP6_ERR_UNSUPPORTED_SHAPE;
+  if (N == 0) return FP6_OK;
+  if (N > INT32_MAX) return FP6_ERR_UNSUPPORTED_SHAPE;
+  if (!scales || (K > 0 && (!W || !q || !pos))) return FP6_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(q) || !aligned16(pos) || !aligned16(scales)) return FP6_ERR_MISALIGNED;
+  const unsigned int zero = 0;
+  cudaError_t e = cudaMemcpyToSymbolAsync(fp6::g_quant_error, &zero, sizeof(zero), 0,
+                                          cudaMemcpyHostToDevice, stream);
+  if (e != cudaSuccess) return FP6_ERR_CUDA;
+  fp6::s24_quantize_kernel<256><<<static_cast<unsigned int>(N), 256, 0, stream>>>(W, K, q, pos, scales);
+  if (cudaGetLastError() != cudaSuccess) return FP6_ERR_CUDA;
+  unsigned int flags = 0;
+  e = cudaMemcpyFromSymbolAsync(&flags, fp6::g_quant_error, sizeof(flags), 0, cudaMemcpyDeviceToHost, stream);
+  if (e != cudaSuccess) return FP6_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return FP6_ERR_CUDA;
+  if (flags & fp6::kQuantNonfinite) return FP6_ERR_NONFINITE;
+  if (flags & fp6::kQuantScaleRange) return FP6_ERR_SCALE_RANGE;
+  return FP6_OK;
+}
+
+fp6_status s24_prepack(const int8_t* q, const uint8_t* pos, int64_t N, int64_t K, void* packed,
+                       size_t packed_bytes, cudaStream_t stream) {
+  fp6_status st = check_shape(N, K);
+  if (st != FP6_OK) return st;
+  if (N == 0 || K == 0) return FP6_OK;
+  if (!q || !pos || !packed) return FP6_ERR_INVALID_ARG;
+  if (packed_bytes < packed_bytes_of(Fmt::S24, N, K)) return FP6_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(pos) || !aligned16(packed)) return FP6_ERR_MISALIGNED;
+  const int64_t work = N * (K / fp6::kTileCols);
+  const int64_t blocks = (work + 255) / 256;
+  fp6::s24_prepack_kernel<<<static_cast<unsigned int>(blocks), 256, 0, stream>>>(q, pos, N, K,
+                                                                                   static_cast<uint8_t*>(packed));
+  return cuda_status(cudaGetLastError());
+}
+
+fp6_status s24_dequant(const void* packed, const uint16_t* scales, int64_t N, int64_t K, uint16_t* W16,
+                       cudaStream_t stream) {
+  return dequant_impl<Fmt::S24>(packed, scales, N, K, W16, stream);
+}
+
+fp6_status s24_linear(const uint16_t* x, const void* packed, const uint16_t* scales, int64_t M, int64_t N,
+                      int64_t K, uint16_t* y, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  return linear_impl<Fmt::S24>(x, packed, scales, M, N, K, y, workspace, workspace_bytes, stream);
 }
 
 fp6_status fp6_get_device_status(cudaStream_t stream) {

@@ -147,7 +147,12 @@ __device__ __forceinline__ uint8_t e3m2_code(float w, float s) {
 //             the low nibbles, right for the high ones) puts four top pieces
 //             in bits 5..2 of four bytes, and Q shifted by 2v-1 (2v) puts
 //             their low bits in bit 1: the e2m3 codes, ready to convert.
-enum class Fmt : int { E3M2 = 0, E2M3 = 1, E2M1 = 2, E2M2 = 3 };
+enum class Fmt : int { E3M2 = 0, E2M3 = 1, E2M1 = 2, E2M2 = 3, S24 = 4 };
+
+// Per-thread state a format's rebuild needs besides the packed words, made
+// once by make_aux() (by every lane of a warp, since the 2:4 format's rebuild
+// reads it across lanes).  The float formats need none.
+struct NoAux {};
 
 // Store a row's words into a tile laid out as 2048-byte blocks of 16 bytes
 // per row (first 4*(W/4) words), then, for W = 10, one 1024-byte block of
@@ -184,6 +189,8 @@ struct Format;
 
 template <>
 struct Format<Fmt::E3M2> {
+  using Aux = NoAux;
+  __device__ static Aux make_aux() { return {}; }
   static constexpr int kTileBytes = 6144;
   static constexpr int kRowWords = 12;
   static constexpr int kMags = 32;          // magnitudes; the sign bit is kMags
@@ -197,6 +204,8 @@ struct Format<Fmt::E3M2> {
 
 template <>
 struct Format<Fmt::E2M3> {
+  using Aux = NoAux;
+  __device__ static Aux make_aux() { return {}; }
   static constexpr int kTileBytes = 6144;
   static constexpr int kRowWords = 12;
   static constexpr int kMags = 32;
@@ -222,6 +231,8 @@ struct Format<Fmt::E2M3> {
 
 template <>
 struct Format<Fmt::E2M1> {
+  using Aux = NoAux;
+  __device__ static Aux make_aux() { return {}; }
   static constexpr int kTileBytes = 4096;
   static constexpr int kRowWords = 8;
   static constexpr int kMags = 8;
@@ -260,6 +271,8 @@ struct Format<Fmt::E2M1> {
 
 template <>
 struct Format<Fmt::E2M2> {
+  using Aux = NoAux;
+  __device__ static Aux make_aux() { return {}; }
   static constexpr int kTileBytes = 5120;
   static constexpr int kRowWords = 10;
   static constexpr int kMags = 16;
@@ -308,6 +321,85 @@ struct Format<Fmt::E2M2> {
   }
   __device__ static void store(uint8_t* tile, int r, const uint32_t (&F)[kRowWords]) { store_row_words(tile, r, F); }
 };
+
+// ---- 2:4 sparse INT4 (Sparse-Marlin) ----------------------------------------
+// In each group of four consecutive weights of a row two are kept; each kept
+// weight is a signed 4-bit code q (two's complement, -8..7) and its value is
+// scale * q.  Tiles of 128 rows x 64 columns in 3072 bytes: row r owns four
+// code words V_w at byte r*16 + 4w and two position words P_h at byte
+// 2048 + r*8 + 4h.  Group j (0..15) of the tile row keeps its two codes in
+// byte j%4 of V_{j/4} (the first kept weight in the low nibble) and its two
+// positions i0 < i1 in bits 4(j%8) .. 4(j%8)+3 of P_{j/8} (i0 in the low two
+// bits).
+//
+// Rebuild of a group: the two nibbles go into the low bits of two fp16 words
+// 0x6400 | (q ^ 8), i.e. 1024 + q + 8, and one half-precision subtraction of
+// 1032 leaves q exactly.  The pair is then placed at positions i0 and i1 of
+// the group's four columns by two byte permutes, whose selectors depend on
+// the position nibble alone: lane l of every warp holds the selectors of
+// nibble l % 16 (make_aux), and a shuffle fetches those of the group's nibble.
+template <>
+struct Format<Fmt::S24> {
+  static constexpr int kTileBytes = 3072;
+  static constexpr int kRowWords = 6;       // V_0..V_3, P_0, P_1
+  struct Aux {
+    uint32_t sel;   // low 16 bits: selector of columns 0,1; high: columns 2,3
+  };
+  __device__ static Aux make_aux() {
+    const int m = static_cast<int>(threadIdx.x & 15);
+    const int i0 = m & 3, i1 = m >> 2;
+    uint32_t sel = 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      // column k takes half 0 (first kept code), half 1 (second) or half 2
+      // (bytes 4, 5: the permute's second operand, zero)
+      const uint32_t h = (k == i0) ? 0u : (k == i1) ? 1u : 2u;
+      sel |= ((2 * h) | ((2 * h + 1) << 4)) << (8 * k);
+    }
+    return {sel};
+  }
+  __device__ static void load(const uint8_t* tile, int r, uint32_t (&F)[kRowWords]) {
+    const uint4 v = *reinterpret_cast<const uint4*>(tile + r * 16);
+    const uint2 q = *reinterpret_cast<const uint2*>(tile + 2048 + r * 8);
+    F[0] = v.x;
+    F[1] = v.y;
+    F[2] = v.z;
+    F[3] = v.w;
+    F[4] = q.x;
+    F[5] = q.y;
+  }
+  __device__ static void rebuild(const uint32_t (&F)[kRowWords], uint32_t (&out)[32], const Aux& aux) {
+    const __half2 k1032 = __halves2half2(__ushort_as_half(0x6408u), __ushort_as_half(0x6408u));
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const uint32_t lo = F[w] & 0x0F0F0F0Fu;           // first kept code of each group
+      const uint32_t hi = (F[w] >> 4) & 0x0F0F0F0Fu;    // second
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const int j = 4 * w + b;
+        uint32_t h = __byte_perm(lo, hi, b | (b << 4) | ((4 + b) << 8) | ((4 + b) << 12));
+        h = (h & 0x000F000Fu) ^ 0x64086408u;
+        const __half2 v = __hsub2(*reinterpret_cast<const __half2*>(&h), k1032);
+        const uint32_t vb = *reinterpret_cast<const uint32_t*>(&v);
+        const uint32_t sel = __shfl_sync(0xffffffffu, aux.sel, static_cast<int>(F[4 + (j >> 3)] >> (4 * (j & 7))), 16);
+        out[2 * j] = __byte_perm(vb, 0u, sel);
+        out[2 * j + 1] = __byte_perm(vb, 0u, sel >> 16);
+      }
+    }
+  }
+};
+
+// Rebuild through a format's per-thread state (the float formats have none).
+template <Fmt F>
+__device__ __forceinline__ void rebuild_row(const uint32_t (&W)[Format<F>::kRowWords], uint32_t (&out)[32],
+                                            const typename Format<F>::Aux& aux) {
+  if constexpr (F == Fmt::S24) {
+    Format<F>::rebuild(W, out, aux);
+  } else {
+    (void)aux;
+    Format<F>::rebuild(W, out);
+  }
+}
 
 // Code of w for the scale s > 0 in format F: |w|/s rounded to the nearest
 // magnitude, ties to the even code, saturating at the largest; sign copied

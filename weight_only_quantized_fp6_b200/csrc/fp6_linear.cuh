@@ -344,6 +344,7 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
     const int quad = warp & 3;               // TMEM lanes 32*quad .. 32*quad+31
     const int r = quad * 32 + lane;          // weight row within the tile
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const auto aux = Fm::make_aux();
     for (int li = g; li < n_local; li += kDeqGroups) {
       const int sw = li % kSW;
       const int s = li % kR;
@@ -354,7 +355,7 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
       for (int t = 0; t < T; ++t) {
         uint32_t Fw[Fm::kRowWords], w[32];
         Fm::load(wst + t * Fm::kTileBytes, r, Fw);
-        Fm::rebuild(Fw, w);
+        rebuild_row<F>(Fw, w, aux);
         tmem_st_32x32b_x32(tmem + lane_base + s * S::kSlotCols + t * 32, w);
       }
       __syncwarp();

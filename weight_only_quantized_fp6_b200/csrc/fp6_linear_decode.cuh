@@ -258,6 +258,7 @@ __global__ void __launch_bounds__(DecodeShape<NCOL, F>::kThreads, 1)
     const int quad = warp & 3;               // TMEM lanes 32*quad .. 32*quad+31
     const int r = quad * 32 + lane;          // weight row within the tile
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const auto aux = Fm::make_aux();
     bool ok = true;
     int j = 0;                               // this group's steps so far
     for (int li = g; li < n_local; li += S::kGroups, ++j) {
@@ -274,10 +275,10 @@ __global__ void __launch_bounds__(DecodeShape<NCOL, F>::kThreads, 1)
         uint32_t F0[Fm::kRowWords], F1[Fm::kRowWords], w[32];
         Fm::load(wst, r, F0);
         if (T > 1) Fm::load(wst + Fm::kTileBytes, r, F1);
-        Fm::rebuild(F0, w);
+        rebuild_row<F>(F0, w, aux);
         tmem_st_32x32b_x32(tmem + lane_base + slot * S::kSlotCols, w);
         if (T > 1) {
-          Fm::rebuild(F1, w);
+          rebuild_row<F>(F1, w, aux);
           tmem_st_32x32b_x32(tmem + lane_base + slot * S::kSlotCols + 32, w);
         }
       }
