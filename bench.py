@@ -39,8 +39,8 @@ UNIT = "GB/s"
 
 
 # bytes per weight of each packed format
-FORMAT_BYTES = {"e3m2": 0.75, "e2m3": 0.75, "e2m1": 0.5, "e2m2": 0.625}
-FORMAT_CODE = {"e3m2": None, "e2m3": 1, "e2m1": 2, "e2m2": 3}
+FORMAT_BYTES = {"e3m2": 0.75, "e2m3": 0.75, "e2m1": 0.5, "e2m2": 0.625, "s24": 0.375}
+FORMAT_CODE = {"e3m2": None, "e2m3": 1, "e2m1": 2, "e2m2": 3, "s24": 4}
 
 
 def wbytes(N, K, per_weight=0.75):
@@ -261,26 +261,41 @@ PREFILL_SHAPES = [(28672, 8192), (8192, 28672)]   # Llama-70B-shaped gate/up and
 PREFILL_MS = [256, 1024, 4096]
 
 
-def _time_us(fn, stream, reps=10):
-    """Average device time of fn() over `reps` calls on `stream` (after one warm-up call)."""
+def _graph_us(fn, stream, launches, reps=5):
+    """Per-call device time of fn(i): `launches` calls captured in one CUDA
+    graph (i = 0 .. launches-1, so fn can rotate over buffers), one untimed
+    replay, then the median over `reps` timed replays."""
     import torch
     with torch.cuda.stream(stream):
-        fn()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record()
+        fn(0)                                 # eager call first: kernel attributes, cuBLAS handles
+        stream.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for i in range(launches):
+                fn(i)
+        graph.replay()
+        ts = []
         for _ in range(reps):
-            fn()
-        e1.record()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            graph.replay()
+            e1.record()
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1e3 / launches)
     torch.cuda.synchronize()
-    return e0.elapsed_time(e1) * 1e3 / reps
+    del graph
+    return statistics.median(ts)
 
 
 def measure_prefill_and_ablation(dev, stream, peaks, packs, scales, xs):
     """Compute-bound prefill sizes (TFLOP/s against the measured dense bf16/fp16
     peak) and the two-kernel comparison of the pages (separate dequant kernel,
     then a cuBLAS fp16 GEMM) next to the fused kernel and a plain fp16 GEMM
-    (cuBLAS W16A16).  cuBLAS appears only here, as context."""
+    (cuBLAS W16A16).  cuBLAS appears only here, as context.  Every figure is a
+    CUDA-graph replay of several calls (median of 5 replays); outputs are
+    allocated once, outside the graphs; the weights (176 MB per prefill
+    layer, more than L2) are read from HBM by every call."""
     import torch
 
     import weight_only_quantized_fp6_b200 as fp6
@@ -293,43 +308,45 @@ def measure_prefill_and_ablation(dev, stream, peaks, packs, scales, xs):
         layer = fp6.FP6Linear.from_float(W)
         del W
         W16 = fp6.dequant(layer.packed, layer.scales, N, K)
+        W16b = torch.empty_like(W16)
         for M in PREFILL_MS:
             x = torch.randn(M, K, device=dev, generator=gen).half()
             y = torch.empty((M, N), dtype=torch.float16, device=dev)
             ws.get(fp6.workspace_bytes(M, N, K))
-            t = _time_us(lambda: fp6.linear(x, layer.packed, layer.scales, N, K, out=y, workspace=ws), stream)
-            t16 = _time_us(lambda: torch.matmul(x, W16.t()), stream)
-            t2 = _time_us(lambda: torch.matmul(x, fp6.dequant(layer.packed, layer.scales, N, K).t()), stream)
+            n_launch = 8 if M <= 1024 else 4
+            t = _graph_us(lambda i: fp6.linear(x, layer.packed, layer.scales, N, K, out=y, workspace=ws),
+                          stream, n_launch)
+            t16 = _graph_us(lambda i: torch.matmul(x, W16.t(), out=y), stream, n_launch)
+            t2 = _graph_us(lambda i: torch.matmul(x, fp6.dequant(layer.packed, layer.scales, N, K, out=W16b).t(),
+                                                  out=y), stream, n_launch)
             fl = 2.0 * M * N * K
             prefill.append({"N": N, "K": K, "M": M, "us": round(t, 2), "tflops": round(fl / t / 1e6, 1),
                             "frac_of_peak": round(fl / t / 1e6 / peaks["bf16_tflops"], 4)})
             ablation.append({"N": N, "K": K, "M": M, "fused_us": round(t, 2), "dequant_then_gemm_us": round(t2, 2),
                              "cublas_w16a16_us": round(t16, 2)})
-        del layer, W16
-    # decode shape: rotate the packed copies (and the fp16 copies, 134 MB each) past L2
+        # the dequant kernel alone: 0.75 B read + 2 B written per weight
+        td = _graph_us(lambda i: fp6.dequant(layer.packed, layer.scales, N, K, out=W16b), stream, 8)
+        dq_bytes = 0.75 * N * K + 2 * N + 2.0 * N * K
+        ablation.append({"N": N, "K": K, "dequant_us": round(td, 2),
+                         "dequant_gbs": round(dq_bytes / td / 1e3, 1),
+                         "dequant_frac_of_hbm": round(dq_bytes / td / 1e3 / peaks["hbm_gbs"], 4)})
+        del layer, W16, W16b
+    # decode shape: rotate the packed copies (and two fp16 copies, 134 MB each) past L2
     N, K = N_DIM, K_DIM
     W16s = [fp6.dequant(packs[i], scales, N, K) for i in range(2)]
+    W16b = torch.empty_like(W16s[0])
     for M in (1, 16):
         x = xs[M]
-        cnt = [0]
-
-        def fused():
-            cnt[0] += 1
-            fp6.linear(x, packs[cnt[0] % len(packs)], scales, N, K, out=y16)
-
-        def two_kernel():
-            cnt[0] += 1
-            torch.matmul(x, fp6.dequant(packs[cnt[0] % len(packs)], scales, N, K).t())
-
-        def w16():
-            cnt[0] += 1
-            torch.matmul(x, W16s[cnt[0] % 2].t())
-
         y16 = torch.empty((M, N), dtype=torch.float16, device=dev)
-        ablation.append({"N": N, "K": K, "M": M, "fused_us": round(_time_us(fused, stream, 22), 2),
-                         "dequant_then_gemm_us": round(_time_us(two_kernel, stream, 22), 2),
-                         "cublas_w16a16_us": round(_time_us(w16, stream, 22), 2)})
-    del W16s
+        nl = 2 * len(packs)
+        fused = _graph_us(lambda i: fp6.linear(x, packs[i % len(packs)], scales, N, K, out=y16, workspace=ws),
+                          stream, nl)
+        two = _graph_us(lambda i: torch.matmul(x, fp6.dequant(packs[i % len(packs)], scales, N, K, out=W16b).t(),
+                                               out=y16), stream, nl)
+        w16 = _graph_us(lambda i: torch.matmul(x, W16s[i % 2].t(), out=y16), stream, nl)
+        ablation.append({"N": N, "K": K, "M": M, "fused_us": round(fused, 2),
+                         "dequant_then_gemm_us": round(two, 2), "cublas_w16a16_us": round(w16, 2)})
+    del W16s, W16b
     return prefill, ablation
 
 
@@ -491,8 +508,14 @@ def run_fp6(args, world, rank, local):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
     e2e_value = world * e2e_steps * len(MS) * wbytes(N_DIM, K_DIM) / (e2e_ms / 1e3) / 1e9
 
-    prefill, ablation = (measure_prefill_and_ablation(dev, stream, peaks, packs, scales, xs)
-                         if rank == 0 and not args.no_extra else (None, None))
+    prefill = ablation = prefill_clocks = None
+    if rank == 0 and not args.no_extra:
+        psampler = ClockSampler(local)
+        psampler.start()
+        time.sleep(0.3)
+        pmark = psampler.mark()
+        prefill, ablation = measure_prefill_and_ablation(dev, stream, peaks, packs, scales, xs)
+        prefill_clocks = psampler.stop(pmark)
 
     ok = fp6.device_status(dev)
     if ok != 0:
@@ -531,6 +554,8 @@ def run_fp6(args, world, rank, local):
         }
         if prefill is not None:
             line["prefill"] = {"metric": "TFLOP/s, fused kernel, M >= 256 (tensor-bound sizes)",
+                               "method": "CUDA-graph replay of 4-8 calls, median of 5 replays",
+                               "clocks": prefill_clocks,
                                "peak_tflops": peaks["bf16_tflops"],
                                "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json bf16_tflops; fp16 runs at "
                                               f"the bf16 rate)", "runs": prefill}

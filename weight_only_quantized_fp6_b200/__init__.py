@@ -118,14 +118,20 @@ def prepack(codes, fmt=None):
     return packed
 
 
-def dequant(packed, scales, N: int, K: int, fmt=None):
-    """packed -> W16 [N,K] fp16; scales None gives the unscaled code values."""
+def dequant(packed, scales, N: int, K: int, fmt=None, out=None):
+    """packed -> W16 [N,K] fp16 (into `out` when given); scales None gives the
+    unscaled code values."""
     torch = _torch()
     _check_fmt(fmt)
     _need_cuda("packed", packed, torch.uint8, 1)
     if scales is not None:
         _need_cuda("scales", scales, torch.float16, 1)
-    out = torch.empty((N, K), dtype=torch.float16, device=packed.device)
+    if out is None:
+        out = torch.empty((N, K), dtype=torch.float16, device=packed.device)
+    else:
+        _need_cuda("out", out, torch.float16, 2)
+        if tuple(out.shape) != (N, K):
+            raise ValueError(f"out must be [{N}, {K}]")
     sp = scales.data_ptr() if scales is not None else None
     lib = _lib.load()
     if fmt is None:

@@ -302,42 +302,47 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
     constexpr int kSlice = 4 / kISS;
     const int kk0 = warp * kSlice;
     const uint32_t d_tmem = tmem + S::kDCol + warp * NCOL;
-    int sg = 0;
-    int ks = static_cast<int>(s0 - tile_first * KS);
-    for (int li = 0; li < n_local; ++li, ks = (ks + 1 == KS) ? 0 : ks + 1) {
-      const bool seg_first = (li == 0) || (ks == 0);
-      const bool seg_last = (li == n_local - 1) || (ks == KS - 1);
-      const int s = li % kR;
-      const int sx = li % kRX;
-      if (seg_first && sg > 0 && !warp_wait(smem_u32(dempty), (sg - 1) & 1, s_abort)) break;
-      if (!warp_wait(smem_u32(&xfull[sx]), (li / kRX) & 1, s_abort)) break;
-      if (!warp_wait(smem_u32(&afull[s]), (li / kR) & 1, s_abort)) break;
-      if (lane == 0) {
-        tc_fence_after();
-        const uint64_t bdesc0 = smem_desc_sw128(smem_u32(smem + sx * S::kXStage));
-        const uint32_t a0 = tmem + s * S::kSlotCols;
-        for (int t = 0; t < T; ++t) {
-          // B descriptor of tile t: start address advances by kXTile bytes (>> 4)
-          const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(t * (S::kXTile >> 4));
+    // The loop runs in lane 0 alone: a barrier test by one lane costs about
+    // 13 cycles against about 110 for a whole warp, and a warp issues
+    // tcgen05.mma at one per ~50 cycles whichever lanes issue, so per-step
+    // warp-wide waits would cost the tensor pipe its feed.
+    if (lane == 0) {
+      int sg = 0;
+      int ks = static_cast<int>(s0 - tile_first * KS);
+      for (int li = 0; li < n_local; ++li, ks = (ks + 1 == KS) ? 0 : ks + 1) {
+        const bool seg_first = (li == 0) || (ks == 0);
+        const bool seg_last = (li == n_local - 1) || (ks == KS - 1);
+        const int s = li % kR;
+        const int sx = li % kRX;
+        if (seg_first && sg > 0 && !wait_bounded(smem_u32(dempty), (sg - 1) & 1, s_abort)) break;
+        if (!wait_bounded(smem_u32(&xfull[sx]), (li / kRX) & 1, s_abort)) break;
+        if (!wait_bounded(smem_u32(&afull[s]), (li / kR) & 1, s_abort)) break;
+        {
+          tc_fence_after();
+          const uint64_t bdesc0 = smem_desc_sw128(smem_u32(smem + sx * S::kXStage));
+          const uint32_t a0 = tmem + s * S::kSlotCols;
+          for (int t = 0; t < T; ++t) {
+            // B descriptor of tile t: start address advances by kXTile bytes (>> 4)
+            const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(t * (S::kXTile >> 4));
 #pragma unroll
-          for (int j = 0; j < kSlice; ++j) {
-            const int kk = kk0 + j;
-            // K = 16 per MMA: 8 TMEM columns of A, 32 bytes along the swizzled B rows
-            mma_f16_ts(d_tmem, a0 + t * 32 + kk * 8, bdesc + static_cast<uint64_t>(kk * 2), idesc,
-                       (seg_first && t == 0 && j == 0) ? 0u : 1u);
+            for (int j = 0; j < kSlice; ++j) {
+              const int kk = kk0 + j;
+              // K = 16 per MMA: 8 TMEM columns of A, 32 bytes along the swizzled B rows
+              mma_f16_ts(d_tmem, a0 + t * 32 + kk * 8, bdesc + static_cast<uint64_t>(kk * 2), idesc,
+                         (seg_first && t == 0 && j == 0) ? 0u : 1u);
+            }
           }
+          tc_commit(smem_u32(&xempty[sx]));
+          tc_commit(smem_u32(&consumed[s]));
+          if (seg_last) tc_commit(smem_u32(dfull));
         }
-        tc_commit(smem_u32(&xempty[sx]));
-        tc_commit(smem_u32(&consumed[s]));
-        if (seg_last) tc_commit(smem_u32(dfull));
+        if (seg_last) ++sg;
       }
-      __syncwarp();
-      if (seg_last) ++sg;
+      // All issued MMAs have finished before TMEM is released.
+      tc_commit(smem_u32(done));
+      wait_bounded(smem_u32(done), 0, s_never);
     }
-    // All issued MMAs have finished before TMEM is released.
-    if (lane == 0) tc_commit(smem_u32(done));
     __syncwarp();
-    warp_wait(smem_u32(done), 0, s_never);
   } else if (warp >= kFirstDeqWarp) {
     // ---------------- dequant warpgroups ----------------
     const int g = (warp - kFirstDeqWarp) >> 2;
