@@ -47,6 +47,7 @@ typedef enum {
     FP6_ERR_NONFINITE = 4,         /* fp6_quantize met a NaN or infinite weight */
     FP6_ERR_SCALE_RANGE = 5,       /* fp6_quantize: max|w|/28 overflows or underflows fp16 */
     FP6_ERR_WORKSPACE = 6,         /* workspace missing or smaller than required */
+    FP6_ERR_LAYOUT_VERSION = 7,    /* a stored packed blob's header does not match this library's layout */
     FP6_ERR_CUDA = 8,              /* a CUDA runtime call or launch failed */
     FP6_ERR_TIMEOUT = 9            /* a kernel's bounded wait ran out (see fp6_get_device_status) */
 } fp6_status;
@@ -228,7 +229,9 @@ fp6_status fp6_linear_plan_for_sms(int64_t M, int64_t N, int64_t K, int sms, int
  * output, ignored on input).  An unknown fmt returns FP6_ERR_INVALID_ARG
  * (fpx_packed_bytes returns 0).
  */
-typedef enum { FPX_E3M2 = 0, FPX_E2M3 = 1, FPX_E2M1 = 2, FPX_E2M2 = 3 } fpx_format;
+typedef enum { FPX_E3M2 = 0, FPX_E2M3 = 1, FPX_E2M1 = 2, FPX_E2M2 = 3,
+               FPX_S24 = 4 /* the 2:4 sparse INT4 format: header functions only (compute via s24_*) */
+} fpx_format;
 
 size_t fpx_packed_bytes(fpx_format fmt, int64_t N, int64_t K);
 fp6_status fpx_quantize(fpx_format fmt, const float *W, int64_t N, int64_t K,
@@ -289,6 +292,47 @@ fp6_status s24_dequant(const void *packed, const uint16_t *scales, int64_t N, in
 fp6_status s24_linear(const uint16_t *x, const void *packed, const uint16_t *scales,
                       int64_t M, int64_t N, int64_t K, uint16_t *y,
                       void *workspace, size_t workspace_bytes, struct CUstream_st *stream);
+
+/*
+ * Stored packed weights.  The TC-FPx article's weights are pre-packed once,
+ * before inference, so a packed buffer is typically written to disk and read
+ * back by a later process, perhaps of another version of this library.  The
+ * device buffers the kernels read carry no header (their layout is fixed by
+ * the entry points above); a stored blob is the 64-byte header below, then
+ * the fp16 scales (2*N bytes), then the packed bytes.  The header records
+ * what the bytes are, so a blob packed under another layout is rejected
+ * instead of being decoded wrongly.
+ *
+ * Header (little-endian; FP6_PACKED_HEADER_BYTES = 64):
+ *   bytes  0.. 3  magic "FP6W"
+ *   bytes  4.. 7  uint32 layout version of the format (FP6_LAYOUT_VERSION_*)
+ *   bytes  8..11  uint32 format (fpx_format, FPX_S24 for the 2:4 format)
+ *   bytes 12..15  uint32 header bytes (64)
+ *   bytes 16..23  int64 N          bytes 24..31  int64 K
+ *   bytes 32..35  uint32 tile rows (128)     bytes 36..39  uint32 tile columns (64)
+ *   bytes 40..43  uint32 bytes per packed tile
+ *   bytes 44..47  uint32 bytes per row scale (2: fp16)
+ *   bytes 48..55  uint64 packed bytes (fpx_packed_bytes / s24_packed_bytes)
+ *   bytes 56..63  zero
+ */
+#define FP6_PACKED_HEADER_BYTES 64
+#define FP6_LAYOUT_VERSION_E3M2 2   /* also FPX_E2M3: whole codes in byte containers, cut codes in top bits */
+#define FP6_LAYOUT_VERSION_E2M1 1
+#define FP6_LAYOUT_VERSION_E2M2 1
+#define FP6_LAYOUT_VERSION_S24 1
+
+/* Writes the header of an N x K weight in format fmt into `header` (HOST
+ * memory, FP6_PACKED_HEADER_BYTES bytes).  FP6_ERR_INVALID_ARG for a NULL
+ * header or an unknown format, FP6_ERR_UNSUPPORTED_SHAPE for a shape the
+ * format cannot pack.  No CUDA call. */
+fp6_status fp6_packed_header(fpx_format fmt, int64_t N, int64_t K, void *header);
+
+/* Checks a stored header (HOST memory) against what this library would write
+ * for (fmt, N, K): FP6_OK if it matches in every field; FP6_ERR_LAYOUT_VERSION
+ * if the magic, the header size, the layout version, the format, the shape,
+ * the tile geometry or the payload size differ; FP6_ERR_INVALID_ARG for a NULL
+ * header or an unknown format.  No CUDA call. */
+fp6_status fp6_packed_header_check(const void *header, fpx_format fmt, int64_t N, int64_t K);
 
 #ifdef __cplusplus
 }

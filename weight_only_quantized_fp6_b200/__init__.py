@@ -23,7 +23,8 @@ from . import _lib
 
 __all__ = ["quantize", "prepack", "dequant", "linear", "linear_plan", "workspace_bytes",
            "packed_bytes", "device_status", "FP6Linear", "FP6Error", "Workspace",
-           "s24_quantize", "s24_prepack", "E3M2", "E2M3", "E2M1", "E2M2", "S24"]
+           "s24_quantize", "s24_prepack", "packed_header", "check_packed_header",
+           "E3M2", "E2M3", "E2M1", "E2M2", "S24"]
 
 FP6Error = _lib.FP6Error
 
@@ -259,6 +260,28 @@ def device_status(device=None) -> int:
     return int(_lib.load().fp6_get_device_status(ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)))
 
 
+HEADER_BYTES = 64
+
+
+def packed_header(N: int, K: int, fmt=None) -> bytes:
+    """The 64-byte header of a stored N x K packed weight (include/fp6.h)."""
+    _check_fmt(fmt)
+    buf = ctypes.create_string_buffer(HEADER_BYTES)
+    _lib.check(_lib.load().fp6_packed_header(E3M2 if fmt is None else fmt, N, K, buf), "fp6_packed_header")
+    return buf.raw
+
+
+def check_packed_header(header: bytes, N: int, K: int, fmt=None) -> None:
+    """Raises FP6Error(FP6_ERR_LAYOUT_VERSION) unless `header` is what this
+    library writes for an N x K weight in `fmt`."""
+    _check_fmt(fmt)
+    if len(header) < HEADER_BYTES:
+        raise FP6Error(7, "fp6_packed_header_check")
+    buf = ctypes.create_string_buffer(bytes(header[:HEADER_BYTES]), HEADER_BYTES)
+    _lib.check(_lib.load().fp6_packed_header_check(buf, E3M2 if fmt is None else fmt, N, K),
+               "fp6_packed_header_check")
+
+
 class FP6Linear:
     """A linear layer whose weight is stored pre-packed (FP6 e3m2 unless `fmt`
     says otherwise) plus fp16 row scales."""
@@ -279,3 +302,39 @@ class FP6Linear:
     def __call__(self, x, out=None):
         return linear(x, self.packed, self.scales, self.N, self.K, out=out, workspace=self.workspace,
                       fmt=self.fmt)
+
+    def save(self, path) -> None:
+        """Writes the layer as a stored blob: the 64-byte header, the fp16
+        scales, the packed bytes."""
+        torch = _torch()
+        with open(path, "wb") as f:
+            f.write(packed_header(self.N, self.K, self.fmt))
+            f.write(self.scales.cpu().view(torch.int16).numpy().tobytes())
+            f.write(self.packed.cpu().numpy().tobytes())
+
+    @classmethod
+    def load(cls, path, device="cuda"):
+        """Reads a blob written by save(); raises FP6Error(FP6_ERR_LAYOUT_VERSION)
+        when its header is not what this library writes for the shape and
+        format it names (for example a blob packed under another layout)."""
+        import struct
+        import numpy as np
+        torch = _torch()
+        with open(path, "rb") as f:
+            header = f.read(HEADER_BYTES)
+            if len(header) < HEADER_BYTES or header[:4] != b"FP6W":
+                raise FP6Error(7, "FP6Linear.load")
+            fmt_code, = struct.unpack_from("<I", header, 8)
+            N, K = struct.unpack_from("<qq", header, 16)
+            fmt = None if fmt_code == E3M2 else int(fmt_code)
+            if fmt not in (None, E2M3, E2M1, E2M2, S24):
+                raise FP6Error(7, "FP6Linear.load")
+            check_packed_header(header, N, K, fmt)
+            scales = np.frombuffer(f.read(2 * N), dtype=np.int16)
+            nbytes = packed_bytes(N, K, fmt)
+            packed = np.frombuffer(f.read(nbytes), dtype=np.uint8)
+            if scales.size != N or packed.size != nbytes:
+                raise FP6Error(7, "FP6Linear.load")
+        dev = torch.device(device)
+        return cls(torch.from_numpy(packed.copy()).to(dev),
+                   torch.from_numpy(scales.copy()).to(dev).view(torch.float16), N, K, fmt)

@@ -15,7 +15,8 @@ LIB_PATH = os.path.join(PKG, "libfp6.so")
 
 STATUS = {
     0: "FP6_OK", 1: "FP6_ERR_INVALID_ARG", 2: "FP6_ERR_UNSUPPORTED_SHAPE", 3: "FP6_ERR_MISALIGNED",
-    4: "FP6_ERR_NONFINITE", 5: "FP6_ERR_SCALE_RANGE", 6: "FP6_ERR_WORKSPACE", 8: "FP6_ERR_CUDA",
+    4: "FP6_ERR_NONFINITE", 5: "FP6_ERR_SCALE_RANGE", 6: "FP6_ERR_WORKSPACE", 7: "FP6_ERR_LAYOUT_VERSION",
+    8: "FP6_ERR_CUDA",
     9: "FP6_ERR_TIMEOUT",
 }
 
@@ -47,6 +48,8 @@ SIGNATURES = {
     "s24_prepack": (_ST, [_P, _P, _I64, _I64, _P, _SZ, _P]),
     "s24_dequant": (_ST, [_P, _P, _I64, _I64, _P, _P]),
     "s24_linear": (_ST, [_P, _P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
+    "fp6_packed_header": (_ST, [_ST, _I64, _I64, _P]),
+    "fp6_packed_header_check": (_ST, [_P, _ST, _I64, _I64]),
 }
 
 _lock = threading.Lock()

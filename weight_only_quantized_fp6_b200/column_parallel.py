@@ -22,7 +22,7 @@ TILE_ROWS = 128
 
 # bytes per weight of each packed format (None = FP6 e3m2, as fp6_*)
 _BYTES_PER_WEIGHT = {None: Fraction(3, 4), 0: Fraction(3, 4), 1: Fraction(3, 4), 2: Fraction(1, 2),
-                     3: Fraction(5, 8)}
+                     3: Fraction(5, 8), 4: Fraction(3, 8)}
 
 
 def shard_rows(N: int, world: int, rank: int) -> tuple[int, int]:
@@ -43,7 +43,7 @@ def packed_range(K: int, n0: int, n1: int, fmt=None) -> tuple[int, int]:
     """Byte range [b0, b1) of rows [n0, n1) inside the packed buffer of an
     N x K weight: every format stores its 128-row tiles one after another, so
     whole row tiles are one contiguous range (0.75 bytes per weight for the
-    6-bit formats, 0.625 for FP5, 0.5 for FP4)."""
+    6-bit formats, 0.625 for FP5, 0.5 for FP4, 0.375 for 2:4 sparse INT4)."""
     if n0 % TILE_ROWS or n1 % TILE_ROWS or K % 64:
         raise ValueError("rows must be whole 128-row tiles and K a multiple of 64")
     if fmt not in _BYTES_PER_WEIGHT:

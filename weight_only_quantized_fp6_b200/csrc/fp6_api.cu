@@ -6,6 +6,7 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -50,6 +51,37 @@ fp6_status check_shape(int64_t N, int64_t K) {
 }
 
 fp6_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FP6_OK : FP6_ERR_CUDA; }
+
+// ---- host-side fault injection (tests of the error paths; no GPU fault) ------
+// FP6_FAULT_INJECT=<point>[:<count>] makes the named host step report failure
+// the next <count> times it runs (every time without a count), as if the CUDA
+// call behind it had failed: "encode" (the activation tensor map), "launch"
+// (a kernel launch: nothing is enqueued), "sync" (the quantizer's stream
+// synchronisation).  The caller sees FP6_ERR_CUDA; no kernel is started.
+struct FaultPlan {
+  char point[16] = {0};
+  long long left = 0;   // < 0: unlimited
+};
+FaultPlan g_fault;
+std::once_flag g_fault_once;
+std::mutex g_fault_mu;
+
+bool fault(const char* point) {
+  std::call_once(g_fault_once, [] {
+    const char* v = std::getenv("FP6_FAULT_INJECT");
+    if (!v || !*v) return;
+    const char* colon = std::strchr(v, ':');
+    const size_t n = colon ? static_cast<size_t>(colon - v) : std::strlen(v);
+    if (n == 0 || n >= sizeof(g_fault.point)) return;
+    std::memcpy(g_fault.point, v, n);
+    g_fault.left = colon ? std::atoll(colon + 1) : -1;
+  });
+  if (g_fault.point[0] == 0 || std::strcmp(g_fault.point, point) != 0) return false;
+  std::lock_guard<std::mutex> lk(g_fault_mu);
+  if (g_fault.left == 0) return false;
+  if (g_fault.left > 0) --g_fault.left;
+  return true;
+}
 
 // ---- per-device cached properties ------------------------------------------
 struct DeviceInfo {
@@ -206,7 +238,7 @@ fp6_status launch_linear(const CUtensorMap& map, const fp6::LinearParams& prm, c
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, map, prm) != cudaSuccess) return FP6_ERR_CUDA;
+  if (fault("launch") || cudaLaunchKernelEx(&cfg, kern, map, prm) != cudaSuccess) return FP6_ERR_CUDA;
   return cuda_status(cudaGetLastError());
 }
 
@@ -234,7 +266,7 @@ fp6_status launch_wave(const CUtensorMap& map, const fp6::LinearParams& prm, cud
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, map, prm) != cudaSuccess) return FP6_ERR_CUDA;
+  if (fault("launch") || cudaLaunchKernelEx(&cfg, kern, map, prm) != cudaSuccess) return FP6_ERR_CUDA;
   return cuda_status(cudaGetLastError());
 }
 
@@ -262,7 +294,7 @@ fp6_status launch_decode(const CUtensorMap& map, const fp6::LinearParams& prm, c
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, map, prm) != cudaSuccess) return FP6_ERR_CUDA;
+  if (fault("launch") || cudaLaunchKernelEx(&cfg, kern, map, prm) != cudaSuccess) return FP6_ERR_CUDA;
   return cuda_status(cudaGetLastError());
 }
 
@@ -300,7 +332,8 @@ fp6_status quantize_impl(const float* W, int64_t N, int64_t K, uint8_t* codes, u
   unsigned int flags = 0;
   e = cudaMemcpyFromSymbolAsync(&flags, fp6::g_quant_error, sizeof(flags), 0, cudaMemcpyDeviceToHost, stream);
   if (e != cudaSuccess) return FP6_ERR_CUDA;
-  if (cudaStreamSynchronize(stream) != cudaSuccess) return FP6_ERR_CUDA;
+  // (the synchronisation itself always runs: the flag copy above writes into `flags`)
+  if (cudaStreamSynchronize(stream) != cudaSuccess || fault("sync")) return FP6_ERR_CUDA;
   if (flags & fp6::kQuantNonfinite) return FP6_ERR_NONFINITE;
   if (flags & fp6::kQuantScaleRange) return FP6_ERR_SCALE_RANGE;
   return FP6_OK;
@@ -395,7 +428,7 @@ fp6_status linear_impl(const uint16_t* x, const void* packed, const uint16_t* sc
   const CUresult cr = encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<uint16_t*>(x), dims, strides, box,
                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (cr != CUDA_SUCCESS) return FP6_ERR_CUDA;
+  if (cr != CUDA_SUCCESS || fault("encode")) return FP6_ERR_CUDA;
 
   switch (pl.ncol) {
     case 16: return launch_decode<16, F>(map, prm, stream, dev);
@@ -419,6 +452,7 @@ const char* fp6_status_string(fp6_status s) {
     case FP6_ERR_NONFINITE: return "FP6_ERR_NONFINITE";
     case FP6_ERR_SCALE_RANGE: return "FP6_ERR_SCALE_RANGE";
     case FP6_ERR_WORKSPACE: return "FP6_ERR_WORKSPACE";
+    case FP6_ERR_LAYOUT_VERSION: return "FP6_ERR_LAYOUT_VERSION";
     case FP6_ERR_CUDA: return "FP6_ERR_CUDA";
     case FP6_ERR_TIMEOUT: return "FP6_ERR_TIMEOUT";
   }
@@ -578,7 +612,8 @@ fp6_status s24_quantize(const float* W, int64_t N, int64_t K, int8_t* q, uint8_t
   unsigned int flags = 0;
   e = cudaMemcpyFromSymbolAsync(&flags, fp6::g_quant_error, sizeof(flags), 0, cudaMemcpyDeviceToHost, stream);
   if (e != cudaSuccess) return FP6_ERR_CUDA;
-  if (cudaStreamSynchronize(stream) != cudaSuccess) return FP6_ERR_CUDA;
+  // (the synchronisation itself always runs: the flag copy above writes into `flags`)
+  if (cudaStreamSynchronize(stream) != cudaSuccess || fault("sync")) return FP6_ERR_CUDA;
   if (flags & fp6::kQuantNonfinite) return FP6_ERR_NONFINITE;
   if (flags & fp6::kQuantScaleRange) return FP6_ERR_SCALE_RANGE;
   return FP6_OK;
@@ -607,6 +642,70 @@ fp6_status s24_dequant(const void* packed, const uint16_t* scales, int64_t N, in
 fp6_status s24_linear(const uint16_t* x, const void* packed, const uint16_t* scales, int64_t M, int64_t N,
                       int64_t K, uint16_t* y, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   return linear_impl<Fmt::S24>(x, packed, scales, M, N, K, y, workspace, workspace_bytes, stream);
+}
+
+// ---- stored packed weights: the blob header ------------------------------------
+}  // extern "C"
+
+namespace {
+
+struct HeaderFields {
+  uint32_t version, tile_bytes;
+  size_t payload;
+};
+
+bool header_fields(int fmt, int64_t N, int64_t K, HeaderFields* h) {
+  Fmt f;
+  if (fmt == FPX_S24) {
+    f = Fmt::S24;
+    h->version = FP6_LAYOUT_VERSION_S24;
+  } else if (fmt_of(fmt, &f)) {
+    h->version = (f == Fmt::E2M1) ? FP6_LAYOUT_VERSION_E2M1
+               : (f == Fmt::E2M2) ? FP6_LAYOUT_VERSION_E2M2 : FP6_LAYOUT_VERSION_E3M2;
+  } else {
+    return false;
+  }
+  h->tile_bytes = static_cast<uint32_t>(packed_bytes_of(f, fp6::kTileRows, fp6::kTileCols));
+  h->payload = packed_bytes_of(f, N, K);
+  return true;
+}
+
+void put32(uint8_t* p, uint32_t v) { std::memcpy(p, &v, 4); }
+void put64(uint8_t* p, uint64_t v) { std::memcpy(p, &v, 8); }
+
+}  // namespace
+
+extern "C" {
+
+fp6_status fp6_packed_header(fpx_format fmt, int64_t N, int64_t K, void* header) {
+  if (!header) return FP6_ERR_INVALID_ARG;
+  HeaderFields h;
+  if (!header_fields(fmt, N, K, &h)) return FP6_ERR_INVALID_ARG;
+  const fp6_status st = check_shape(N, K);
+  if (st != FP6_OK) return st;
+  uint8_t* b = static_cast<uint8_t*>(header);
+  std::memset(b, 0, FP6_PACKED_HEADER_BYTES);
+  std::memcpy(b, "FP6W", 4);
+  put32(b + 4, h.version);
+  put32(b + 8, static_cast<uint32_t>(fmt));
+  put32(b + 12, FP6_PACKED_HEADER_BYTES);
+  put64(b + 16, static_cast<uint64_t>(N));
+  put64(b + 24, static_cast<uint64_t>(K));
+  put32(b + 32, fp6::kTileRows);
+  put32(b + 36, fp6::kTileCols);
+  put32(b + 40, h.tile_bytes);
+  put32(b + 44, 2);
+  put64(b + 48, h.payload);
+  return FP6_OK;
+}
+
+fp6_status fp6_packed_header_check(const void* header, fpx_format fmt, int64_t N, int64_t K) {
+  if (!header) return FP6_ERR_INVALID_ARG;
+  uint8_t want[FP6_PACKED_HEADER_BYTES];
+  const fp6_status st = fp6_packed_header(fmt, N, K, want);
+  if (st == FP6_ERR_UNSUPPORTED_SHAPE) return FP6_ERR_LAYOUT_VERSION;   // no blob of this library has that shape
+  if (st != FP6_OK) return st;
+  return std::memcmp(want, header, FP6_PACKED_HEADER_BYTES) == 0 ? FP6_OK : FP6_ERR_LAYOUT_VERSION;
 }
 
 fp6_status fp6_get_device_status(cudaStream_t stream) {
