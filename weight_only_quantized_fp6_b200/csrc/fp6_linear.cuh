@@ -439,22 +439,26 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
         if (lane == 0) mbar_arrive(eb);
         if (!warp_wait(eb, 1, s_abort)) break;
         if (s_last[which]) {
-          for (int c0 = 0; c0 < mcount; c0 += 8) {
-            float acc[8];
+          // kSumCols columns of one contributor per step: their loads are all
+          // in flight together, so a tile costs about (NCOL / kSumCols) x
+          // contributors L2 round trips rather than one per 8 columns.
+          constexpr int kSumCols = NCOL < 32 ? NCOL : 32;
+          for (int c0 = 0; c0 < mcount; c0 += kSumCols) {
+            float acc[kSumCols];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
+            for (int j = 0; j < kSumCols; ++j) acc[j] = 0.0f;
             for (int cc = c_lo; cc <= c_hi; ++cc) {
               const float* src = p.partials +
                                  static_cast<long long>(partial_slot(cc, tile, total, G, KS)) * NCOL * 128 +
                                  c0 * 128 + r;
-              float v[8];
+              float v[kSumCols];
 #pragma unroll
-              for (int j = 0; j < 8; ++j) v[j] = __ldcg(src + j * 128);
+              for (int j = 0; j < kSumCols; ++j) v[j] = __ldcg(src + j * 128);
 #pragma unroll
-              for (int j = 0; j < 8; ++j) acc[j] += v[j];
+              for (int j = 0; j < kSumCols; ++j) acc[j] += v[j];
             }
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
+            for (int j = 0; j < kSumCols; ++j)
               if (c0 + j < mcount)
                 p.y[static_cast<long long>(m0 + c0 + j) * p.N + n] = __half_as_ushort(__float2half_rn(acc[j] * mul));
           }

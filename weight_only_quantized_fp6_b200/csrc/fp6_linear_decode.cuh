@@ -384,14 +384,18 @@ __global__ void __launch_bounds__(DecodeShape<NCOL, F>::kThreads, 1)
         }
       };
       // Partials of contributors c_lo+1 .. c_hi summed in CTA order, columns
-      // c0 .. c0+7.
-      auto others8 = [&](int c0, float (&q)[8]) {
+      // c0 .. c0+15 (those below mcount): one contributor's 16 loads are in
+      // flight together, one L2 round trip per contributor and 16 columns.
+      auto others16 = [&](int c0, float (&q)[16]) {
 #pragma unroll
-        for (int jj = 0; jj < 8; ++jj) q[jj] = 0.0f;
+        for (int jj = 0; jj < 16; ++jj) q[jj] = 0.0f;
         for (int cc = c_lo + 1; cc <= c_hi; ++cc) {
           const float* src = decode_partial<NCOL>(p.partials, 2 * cc, r) + c0 * 128;
+          float v[16];
 #pragma unroll
-          for (int jj = 0; jj < 8; ++jj) q[jj] += __ldcg(src + jj * 128);
+          for (int jj = 0; jj < 16; ++jj) v[jj] = (c0 + jj < mcount) ? __ldcg(src + jj * 128) : 0.0f;
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) q[jj] += v[jj];
         }
       };
       auto store8 = [&](int c0, const float (&v)[8]) {
@@ -434,13 +438,19 @@ __global__ void __launch_bounds__(DecodeShape<NCOL, F>::kThreads, 1)
       auto finish_from_partials = [&]() {
         const float* lo = decode_partial<NCOL>(p.partials, 2 * c_lo + 1, r);
 #pragma unroll
-        for (int c0 = 0; c0 < NCOL; c0 += 8) {
+        for (int c0 = 0; c0 < NCOL; c0 += 16) {
           if (c0 >= mcount) break;
-          float q[8];
-          others8(c0, q);
+          float q[16], v[16];
+          others16(c0, q);
 #pragma unroll
-          for (int jj = 0; jj < 8; ++jj) q[jj] += __ldcg(lo + (c0 + jj) * 128);
-          store8(c0, q);
+          for (int jj = 0; jj < 16; ++jj) v[jj] = (c0 + jj < mcount) ? __ldcg(lo + (c0 + jj) * 128) : 0.0f;
+#pragma unroll
+          for (int h = 0; h < 16; h += 8) {
+            float w[8];
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) w[jj] = q[h + jj] + v[h + jj];
+            store8(c0 + h, w);
+          }
         }
         __syncwarp();
         if (lane == 0) *cnt = 0u;            // every contributor has counted: reset for the next launch
@@ -462,20 +472,15 @@ __global__ void __launch_bounds__(DecodeShape<NCOL, F>::kThreads, 1)
         }
         release();
       } else if (finisher) {
-        // With 16 token columns the others' partials fit in registers: sum
-        // them while this CTA's last MMAs still run, as soon as all are there.
+        // The others' partials, 16 columns at a time.  With 16 token columns
+        // that is all of them: sum them while this CTA's last MMAs still run,
+        // as soon as all are there.
         float pre[16];
         bool pre_ok = false;
         if constexpr (NCOL == 16) {
           while (true) {
             if (all_counted()) {
-#pragma unroll
-              for (int c0 = 0; c0 < 16; c0 += 8) {
-                float q[8];
-                others8(c0, q);
-#pragma unroll
-                for (int jj = 0; jj < 8; ++jj) pre[c0 + jj] = q[jj];
-              }
+              others16(0, pre);
               pre_ok = true;
               break;
             }
@@ -488,23 +493,18 @@ __global__ void __launch_bounds__(DecodeShape<NCOL, F>::kThreads, 1)
         tc_fence_after();
         if (pre_ok || all_counted()) {
 #pragma unroll
-          for (int c0 = 0; c0 < NCOL; c0 += 8) {
+          for (int c0 = 0; c0 < NCOL; c0 += 16) {
             if (c0 >= mcount) break;
-            float acc[8], q[8];
-            own8(c0, acc);
-            if constexpr (NCOL == 16) {
-              if (pre_ok) {
+            if (!pre_ok) others16(c0, pre);
 #pragma unroll
-                for (int jj = 0; jj < 8; ++jj) q[jj] = pre[(c0 + jj) & 15];
-              } else {
-                others8(c0, q);
-              }
-            } else {
-              others8(c0, q);
+            for (int h = 0; h < 16; h += 8) {
+              if (c0 + h >= mcount) break;
+              float acc[8];
+              own8(c0 + h, acc);
+#pragma unroll
+              for (int jj = 0; jj < 8; ++jj) acc[jj] = pre[h + jj] + acc[jj];
+              store8(c0 + h, acc);
             }
-#pragma unroll
-            for (int jj = 0; jj < 8; ++jj) acc[jj] = q[jj] + acc[jj];
-            store8(c0, acc);
           }
           release();
           __syncwarp();
