@@ -7,9 +7,8 @@
 // weights with bit-parallel SIMT work in registers, and overlaps the two with
 // a software pipeline.  On sm_100a this becomes a warp-specialised persistent
 // kernel.  The unit of the pipeline is a "step": T consecutive 64-column tiles
-// of one 128-row weight tile (T = 1, 2 or 4).  Every mbarrier wait or
-// tcgen05.commit costs a warp about 90 cycles and one MMA issue about 50, so
-// per-step synchronisation is amortised over T tiles.
+// of one 128-row weight tile (T = 1, 2 or 4), so that per-step
+// synchronisation is amortised over T tiles.
 //
 //   warp 20       weight producer: one bulk copy of the step's T packed tiles
 //                 (contiguous, T * 6144 bytes) into a smem ring (SW stages);
@@ -28,13 +27,17 @@
 //                 summed in a fixed order, * scale, fp16 store, or the
 //                 split-K partial and fix-up.
 //
-// Three rings: packed weights (SW smem stages, filled by the weight
-// producer, released by the dequant group), x (RX smem stages, released by
-// the issuers' commits) and dequantized weights (R TMEM slots, released by the
-// issuers' commits).  Every mbarrier's consumers wait on its phases in order
-// (a weight stage or TMEM slot always belongs to the same dequant group: SW
-// and R are multiples of the group count), so no wait can alias a phase two
-// steps ahead.
+// Rings: packed weights (SW smem stages, filled by the weight producer,
+// released by the dequant group), x (RX smem stages) and dequantized weights
+// (R TMEM slots).  The MMA issuer is the one serial thread of the pipeline
+// (an MMA issue costs it about 100 cycles, a barrier test or commit 80-130),
+// so it handles one barrier of each kind per step: the step's dequant group
+// waits for the step's x stage to land before it signals "ready", and one
+// commit per step ("freed") releases both the x stage and the TMEM slot.
+// Those two barriers form a ring of L = lcm(R, RX) steps.  Every mbarrier's
+// waiters wait on its phases in order (a weight stage, TMEM slot or step
+// barrier always belongs to the same dequant group: SW, R and L are multiples
+// of the group count), so no wait can alias a phase two steps ahead.
 //
 // Work split: the (token tile, row tile, step) iterations are laid out
 // row-tile major and cut into G contiguous, equal ranges, one per persistent
@@ -74,6 +77,9 @@ constexpr int kMaxGrid = 1024;                // persistent CTAs at most (one pe
 constexpr int kCounterBytes = kMaxGrid * 16;   // up to four counters per CTA
 constexpr uint32_t kTmemCols = 512;
 
+constexpr int gcd_int(int a, int b) { return b == 0 ? a : gcd_int(b, a % b); }
+constexpr int lcm_int(int a, int b) { return a / gcd_int(a, b) * b; }
+
 template <int NCOL, Fmt F = Fmt::E3M2>
 struct LinearShape {
   static_assert(NCOL == 16 || NCOL == 32 || NCOL == 64 || NCOL == 128 || NCOL == 256, "NCOL");
@@ -83,7 +89,7 @@ struct LinearShape {
   static constexpr int kTileBytes = Format<F>::kTileBytes;
   static constexpr int kWStage = kTMax * kTileBytes;
   static constexpr int kIssuers = (NCOL <= 32) ? 4 : (NCOL == 64) ? 2 : 1;
-  static constexpr int kRX = (NCOL == 16) ? 8 : (NCOL <= 64) ? 4 : 3;     // x stages (>= 3)
+  static constexpr int kRX = (NCOL == 16) ? 8 : (NCOL == 32) ? 4 : 3;     // x stages (>= 3)
   // weight stages of 6-bit tiles; the same bytes in FP4 tiles
   static constexpr int kSW = ((NCOL <= 32) ? 6 : (NCOL == 64) ? 12 : (NCOL == 128) ? 9 : 18) * 6144 / kTileBytes /
                              kDeqGroups * kDeqGroups;
@@ -92,11 +98,22 @@ struct LinearShape {
   static constexpr int kDCol = kR * kSlotCols;              // accumulators after the slots
   static constexpr int kWOff = kRX * kXStage;               // weight ring after the x ring
   static constexpr int kBarOff = kWOff + kSW * kWStage;
-  static constexpr int kNumBars = 2 * kSW + 2 * kRX + 2 * kR + 5;
+  // Step barriers, a ring of kL (a multiple of the x stages and of the TMEM
+  // slots): "ready" (the step's dequant group has written its TMEM slot and
+  // seen its x stage land) and "freed" (the step's MMAs have completed).
+  static constexpr int kL = lcm_int(kR, kRX);
+  // wfull, wempty [SW]; xfull [RX]; ready, freed [L]; dfull, dempty, done, epi[2]
+  static constexpr int kNumBars = 2 * kSW + kRX + 2 * kL + 5;
+  // columns per TMEM read in the epilogue: kIssuers reads of kEC 32-bit columns
+  static constexpr int kEC = 32 / kIssuers;
   static constexpr int kBarrierBytes = 1024;
   static constexpr int kSmemBytes = kBarOff + kBarrierBytes + 1024;  // + alignment slack
   static_assert(kXTile % 1024 == 0 && kTileBytes % 1024 == 0, "1024-byte aligned tiles");
   static_assert(kSW % kDeqGroups == 0 && kR % kDeqGroups == 0, "ring slots owned by one group");
+  // A dequant group waiting for step li's x stage finds the stage's previous
+  // fill (step li - RX) complete: it was its own step, or it precedes step
+  // li - R, whose MMAs have completed.  So no parity wait can alias.
+  static_assert(kRX % kDeqGroups == 0 || kRX >= kR, "x stage phases seen in order");
   static_assert(kDCol + kIssuers * NCOL <= static_cast<int>(kTmemCols), "TMEM budget");
   static_assert(kNumBars * 8 + 32 <= kBarrierBytes, "barrier area");
   static_assert(kNumBars <= kLinearThreads, "one thread per barrier at set-up");
@@ -131,6 +148,37 @@ __host__ __device__ __forceinline__ int range_owner(long long i, long long total
 // can be partial).
 __host__ __device__ __forceinline__ int partial_slot(int c, long long t, long long total, int G, int KS) {
   return 2 * c + ((range_begin(c, total, G) / KS == t) ? 0 : 1);
+}
+
+// Rows n of a warp's lanes, columns (tokens) m0 + j, j < C, of y as fp16
+// (v[j] * mul, rounded to nearest even), stored for j < count.  Lanes l and
+// l ^ 1 swap one value per column pair so that each stores two adjacent rows
+// of one token as one 32-bit word.  n is the row of an even lane at l & ~1;
+// y and N keep every such word 4-byte aligned.
+template <int C>
+__device__ __forceinline__ void store_y_pairs(uint16_t* y, const float (&v)[C], float mul, long long m0, int count,
+                                              int N, int n, int lane) {
+  static_assert(C % 2 == 0, "column pairs");
+  const int odd = lane & 1;
+  uint32_t* yw = reinterpret_cast<uint32_t*>(y);
+#pragma unroll
+  for (int j = 0; j < C; j += 2) {
+    const uint32_t ha = __half_as_ushort(__float2half_rn(v[j] * mul));
+    const uint32_t hb = __half_as_ushort(__float2half_rn(v[j + 1] * mul));
+    const uint32_t other = __shfl_xor_sync(0xffffffffu, odd ? ha : hb, 1);
+    const uint32_t lo = odd ? other : ha;       // row n - odd
+    const uint32_t hi = odd ? hb : other;       // row n - odd + 1
+    const int t = j + odd;
+    if (t < count) yw[((m0 + t) * N + (n - odd)) >> 1] = lo | (hi << 16);
+  }
+}
+
+// C 32-bit TMEM columns of the warp's 32 lanes (C = 8, 16 or 32).
+template <int C>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&v)[C]) {
+  if constexpr (C == 32) tmem_ld_32x32b_x32(taddr, v);
+  else if constexpr (C == 16) tmem_ld_32x32b_x16(taddr, v);
+  else tmem_ld_32x32b_x8(taddr, v);
 }
 
 // Every lane of the warp waits; the warp continues only if all lanes saw the
@@ -182,16 +230,17 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
   constexpr int kRX = S::kRX;
   constexpr int kSW = S::kSW;
   constexpr int kISS = S::kIssuers;
+  constexpr int kL = S::kL;
+  constexpr int kEC = S::kEC;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBarOff);
   uint64_t* wfull = bars;
   uint64_t* wempty = wfull + kSW;
-  uint64_t* xfull = wempty + kSW;
-  uint64_t* xempty = xfull + kRX;                 // x stage free (issuer commits)
-  uint64_t* afull = xempty + kRX;
-  uint64_t* consumed = afull + kR;                // TMEM slot free (issuer commits)
-  uint64_t* dfull = consumed + kR;
+  uint64_t* xfull = wempty + kSW;                 // x stage landed (producer arrive + tx)
+  uint64_t* ready = xfull + kRX;                  // step ready (its dequant group)
+  uint64_t* freed = ready + kL;                   // step's MMAs complete (issuer commits)
+  uint64_t* dfull = freed + kL;
   uint64_t* dempty = dfull + 1;
   uint64_t* done = dempty + 1;
   uint64_t* epi = done + 1;                       // [2]: fix-up meeting of the first / last split segment
@@ -221,12 +270,11 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
   // Barrier set-up, one thread per barrier.
   if (threadIdx.x < S::kNumBars) {
     const int b = threadIdx.x;
-    const int bx = 2 * kSW, ba = bx + 2 * kRX, bd = ba + 2 * kR;
+    const int bx = 2 * kSW, br = bx + kRX, bf = br + kL, bd = bf + kL;
     uint32_t count = 1;                                       // wfull, xfull: producer arrive + tx
     if (b >= kSW && b < bx) count = 4;                        // wempty: the reading group's 4 warps
-    else if (b >= bx + kRX && b < ba) count = kISS;           // xempty: issuer commits
-    else if (b >= ba && b < ba + kR) count = 4;               // afull: the writing group
-    else if (b >= ba + kR && b < bd) count = kISS;            // consumed: issuer commits
+    else if (b >= br && b < bf) count = 4;                    // ready: the step's dequant group
+    else if (b >= bf && b < bd) count = kISS;                 // freed: issuer commits
     else if (b == bd) count = kISS;                           // dfull
     else if (b == bd + 1) count = 4;                          // dempty: epilogue warps
     else if (b == bd + 2) count = kISS;                       // done
@@ -285,7 +333,8 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
     int issued = 0;
     for (int li = 0; li < n_local; ++li, cur.next()) {
       const int s = li % kRX;
-      if (li >= kRX && !warp_wait(smem_u32(&xempty[s]), ((li / kRX) - 1) & 1, s_abort)) break;
+      // the stage's previous step (li - RX) has had its MMAs
+      if (li >= kRX && !warp_wait(smem_u32(&freed[(li - kRX) % kL]), ((li - kRX) / kL) & 1, s_abort)) break;
       if (lane == 0) {
         const uint32_t fb = smem_u32(&xfull[s]);
         mbar_arrive_expect_tx(fb, bytes);
@@ -315,8 +364,7 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
         const int s = li % kR;
         const int sx = li % kRX;
         if (seg_first && sg > 0 && !wait_bounded(smem_u32(dempty), (sg - 1) & 1, s_abort)) break;
-        if (!wait_bounded(smem_u32(&xfull[sx]), (li / kRX) & 1, s_abort)) break;
-        if (!wait_bounded(smem_u32(&afull[s]), (li / kR) & 1, s_abort)) break;
+        if (!wait_bounded(smem_u32(&ready[li % kL]), (li / kL) & 1, s_abort)) break;
         {
           tc_fence_after();
           const uint64_t bdesc0 = smem_desc_sw128(smem_u32(smem + sx * S::kXStage));
@@ -332,8 +380,7 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
                          (seg_first && t == 0 && j == 0) ? 0u : 1u);
             }
           }
-          tc_commit(smem_u32(&xempty[sx]));
-          tc_commit(smem_u32(&consumed[s]));
+          tc_commit(smem_u32(&freed[li % kL]));
           if (seg_last) tc_commit(smem_u32(dfull));
         }
         if (seg_last) ++sg;
@@ -354,7 +401,7 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
       const int sw = li % kSW;
       const int s = li % kR;
       if (!warp_wait(smem_u32(&wfull[sw]), (li / kSW) & 1, s_abort)) break;
-      if (li >= kR && !warp_wait(smem_u32(&consumed[s]), ((li / kR) - 1) & 1, s_abort)) break;
+      if (li >= kR && !warp_wait(smem_u32(&freed[(li - kR) % kL]), ((li - kR) / kL) & 1, s_abort)) break;
       tc_fence_after();
       const uint8_t* wst = smem + S::kWOff + sw * S::kWStage;
       for (int t = 0; t < T; ++t) {
@@ -366,9 +413,11 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&wempty[sw]));   // smem fragments read
       tmem_wait_st();
+      // The step's x stage has landed too: the issuer then waits on one barrier.
+      if (!warp_wait(smem_u32(&xfull[li % kRX]), (li / kRX) & 1, s_abort)) break;
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&afull[s]));
+      if (lane == 0) mbar_arrive(smem_u32(&ready[li % kL]));
     }
   } else if (warp >= kEpiWarp && warp < kEpiWarp + 4) {
     // ---------------- epilogue warpgroup: segments in order ----------------
@@ -392,17 +441,22 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
       const bool split = c_lo != c_hi;
       const int which = (tile == tile_first) ? 0 : 1;   // this CTA's first or last segment
       float* part = p.partials + static_cast<long long>(2 * c + which) * NCOL * 128;
-      for (int c0 = 0; c0 < NCOL; c0 += 8) {
-        float acc[8];
+      for (int c0 = 0; c0 < NCOL; c0 += kEC) {
+        // kEC columns of every issuer's accumulator, read together, summed
+        // in issuer order
+        uint32_t v[kISS][kEC];
 #pragma unroll
-        for (int i = 0; i < kISS; ++i) {
-          uint32_t v[8];
-          tmem_ld_32x32b_x8(tmem + lane_base + S::kDCol + i * NCOL + c0, v);
-          tmem_wait_ld();
+        for (int i = 0; i < kISS; ++i) tmem_ld_cols<kEC>(tmem + lane_base + S::kDCol + i * NCOL + c0, v[i]);
+        tmem_wait_ld();
+        float acc[kEC];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) acc[j] = (i == 0) ? __uint_as_float(v[j]) : acc[j] + __uint_as_float(v[j]);
+        for (int j = 0; j < kEC; ++j) {
+          float a = __uint_as_float(v[0][j]);
+#pragma unroll
+          for (int i = 1; i < kISS; ++i) a += __uint_as_float(v[i][j]);
+          acc[j] = a;
         }
-        if (c0 + 8 >= NCOL) {
+        if (c0 + kEC >= NCOL) {
           // accumulators fully read: the next segment may overwrite them
           tc_fence_before();
           __syncwarp();
@@ -410,13 +464,9 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
         }
         if (split) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) __stcg(part + (c0 + j) * 128 + r, acc[j]);
+          for (int j = 0; j < kEC; ++j) __stcg(part + (c0 + j) * 128 + r, acc[j]);
         } else {
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            if (c0 + j < mcount)
-              p.y[static_cast<long long>(m0 + c0 + j) * p.N + n] = __half_as_ushort(__float2half_rn(acc[j] * mul));
-          }
+          store_y_pairs<kEC>(p.y, acc, mul, m0 + c0, mcount - c0, p.N, n, lane);
         }
       }
       if (split) {
@@ -457,10 +507,7 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
 #pragma unroll
               for (int j = 0; j < kSumCols; ++j) acc[j] += v[j];
             }
-#pragma unroll
-            for (int j = 0; j < kSumCols; ++j)
-              if (c0 + j < mcount)
-                p.y[static_cast<long long>(m0 + c0 + j) * p.N + n] = __half_as_ushort(__float2half_rn(acc[j] * mul));
+            store_y_pairs<kSumCols>(p.y, acc, mul, m0 + c0, mcount - c0, p.N, n, lane);
           }
           if (leader) p.counters[c_lo] = 0u;
         }

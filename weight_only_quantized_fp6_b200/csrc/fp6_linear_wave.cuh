@@ -59,16 +59,17 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
   constexpr int kRX = S::kRX;
   constexpr int kSW = S::kSW;
   constexpr int kISS = S::kIssuers;
+  constexpr int kL = S::kL;
+  constexpr int kEC = S::kEC;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBarOff);
   uint64_t* wfull = bars;
   uint64_t* wempty = wfull + kSW;
-  uint64_t* xfull = wempty + kSW;
-  uint64_t* xempty = xfull + kRX;                 // x stage free (issuer commits)
-  uint64_t* afull = xempty + kRX;
-  uint64_t* consumed = afull + kR;                // TMEM slot free (issuer commits)
-  uint64_t* dfull = consumed + kR;
+  uint64_t* xfull = wempty + kSW;                 // x stage landed (producer arrive + tx)
+  uint64_t* ready = xfull + kRX;                  // step ready (its dequant group)
+  uint64_t* freed = ready + kL;                   // step's MMAs complete (issuer commits)
+  uint64_t* dfull = freed + kL;
   uint64_t* dempty = dfull + 1;
   uint64_t* done = dempty + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + S::kNumBars);
@@ -95,12 +96,11 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
   // stay unused here).
   if (threadIdx.x < S::kNumBars) {
     const int b = threadIdx.x;
-    const int bx = 2 * kSW, ba = bx + 2 * kRX, bd = ba + 2 * kR;
+    const int bx = 2 * kSW, br = bx + kRX, bf = br + kL, bd = bf + kL;
     uint32_t count = 1;                                       // wfull, xfull: producer arrive + tx
     if (b >= kSW && b < bx) count = 4;                        // wempty: the reading group's 4 warps
-    else if (b >= bx + kRX && b < ba) count = kISS;           // xempty: issuer commits
-    else if (b >= ba && b < ba + kR) count = 4;               // afull: the writing group
-    else if (b >= ba + kR && b < bd) count = kISS;            // consumed: issuer commits
+    else if (b >= br && b < bf) count = 4;                    // ready: the step's dequant group
+    else if (b >= bf && b < bd) count = kISS;                 // freed: issuer commits
     else if (b == bd) count = kISS;                           // dfull
     else if (b == bd + 1) count = 4;                          // dempty: epilogue warps
     else if (b == bd + 2) count = kISS;                       // done
@@ -154,7 +154,8 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
     int issued = 0;
     for (int li = 0; li < n_local; ++li, cur.next()) {
       const int s = li % kRX;
-      if (li >= kRX && !warp_wait(smem_u32(&xempty[s]), ((li / kRX) - 1) & 1, s_abort)) break;
+      // the stage's previous step (li - RX) has had its MMAs
+      if (li >= kRX && !warp_wait(smem_u32(&freed[(li - kRX) % kL]), ((li - kRX) / kL) & 1, s_abort)) break;
       if (lane == 0) {
         const uint32_t fb = smem_u32(&xfull[s]);
         mbar_arrive_expect_tx(fb, bytes);
@@ -184,8 +185,7 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
         const int s = li % kR;
         const int sx = li % kRX;
         if (seg_first && sg > 0 && !wait_bounded(smem_u32(dempty), (sg - 1) & 1, s_abort)) break;
-        if (!wait_bounded(smem_u32(&xfull[sx]), (li / kRX) & 1, s_abort)) break;
-        if (!wait_bounded(smem_u32(&afull[s]), (li / kR) & 1, s_abort)) break;
+        if (!wait_bounded(smem_u32(&ready[li % kL]), (li / kL) & 1, s_abort)) break;
         {
           tc_fence_after();
           const uint64_t bdesc0 = smem_desc_sw128(smem_u32(smem + sx * S::kXStage));
@@ -199,8 +199,7 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
                          (seg_first && t == 0 && j == 0) ? 0u : 1u);
             }
           }
-          tc_commit(smem_u32(&xempty[sx]));
-          tc_commit(smem_u32(&consumed[s]));
+          tc_commit(smem_u32(&freed[li % kL]));
           if (seg_last) tc_commit(smem_u32(dfull));
         }
         if (seg_last) ++sg;
@@ -221,7 +220,7 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
       const int sw = li % kSW;
       const int s = li % kR;
       if (!warp_wait(smem_u32(&wfull[sw]), (li / kSW) & 1, s_abort)) break;
-      if (li >= kR && !warp_wait(smem_u32(&consumed[s]), ((li / kR) - 1) & 1, s_abort)) break;
+      if (li >= kR && !warp_wait(smem_u32(&freed[(li - kR) % kL]), ((li - kR) / kL) & 1, s_abort)) break;
       tc_fence_after();
       const uint8_t* wst = smem + S::kWOff + sw * S::kWStage;
       for (int t = 0; t < T; ++t) {
@@ -233,9 +232,11 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&wempty[sw]));   // smem fragments read
       tmem_wait_st();
+      // The step's x stage has landed too: the issuer then waits on one barrier.
+      if (!warp_wait(smem_u32(&xfull[li % kRX]), (li / kRX) & 1, s_abort)) break;
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&afull[s]));
+      if (lane == 0) mbar_arrive(smem_u32(&ready[li % kL]));
     }
   } else if (warp >= kEpiWarp && warp < kEpiWarp + 4) {
     // ---------------- epilogue warpgroup: this CTA's tiles in order ----------------
@@ -253,27 +254,26 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
       const int m0 = mt * NCOL;
       const int mcount = min(NCOL, p.M - m0);
       const float mul = __half2float(__ushort_as_half(p.scales[n]));
-      for (int c0 = 0; c0 < NCOL; c0 += 8) {
-        float acc[8];
+      for (int c0 = 0; c0 < NCOL; c0 += kEC) {
+        uint32_t v[kISS][kEC];
 #pragma unroll
-        for (int i = 0; i < kISS; ++i) {
-          uint32_t v[8];
-          tmem_ld_32x32b_x8(tmem + lane_base + S::kDCol + i * NCOL + c0, v);
-          tmem_wait_ld();
+        for (int i = 0; i < kISS; ++i) tmem_ld_cols<kEC>(tmem + lane_base + S::kDCol + i * NCOL + c0, v[i]);
+        tmem_wait_ld();
+        float acc[kEC];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) acc[j] = (i == 0) ? __uint_as_float(v[j]) : acc[j] + __uint_as_float(v[j]);
+        for (int j = 0; j < kEC; ++j) {
+          float a = __uint_as_float(v[0][j]);
+#pragma unroll
+          for (int i = 1; i < kISS; ++i) a += __uint_as_float(v[i][j]);
+          acc[j] = a;
         }
-        if (c0 + 8 >= NCOL) {
+        if (c0 + kEC >= NCOL) {
           // accumulators fully read: the next tile may overwrite them
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_u32(dempty));
         }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (c0 + j < mcount)
-            p.y[static_cast<long long>(m0 + c0 + j) * p.N + n] = __half_as_ushort(__float2half_rn(acc[j] * mul));
-        }
+        store_y_pairs<kEC>(p.y, acc, mul, m0 + c0, mcount - c0, p.N, n, lane);
       }
     }
   }
