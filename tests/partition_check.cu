@@ -1,5 +1,6 @@
 // Host-only check of the persistent-grid work split used by the fused linear
-// kernel (range_begin / range_owner / partial_slot from fp6_linear.cuh).
+// kernel (range_begin / range_owner / partial_slot / split_slot from
+// fp6_linear.cuh).
 // Prints "ok" or the first violated property.  Runs on the CPU.
 #include <cstdio>
 #include <set>
@@ -29,6 +30,7 @@ static int check(long long tiles, int KT, int G) {
     for (int cc = lo; cc <= hi; ++cc) {
       const int s = partial_slot(cc, t, total, G, KT);
       if (s < 0 || s >= 2 * G) return 6;
+      if (split_slot(cc, lo, range_begin(lo, total, G) == t * KT) != s) return 9;   // the kernel's lookup
       if (!slots.insert(s).second) return 7;       // one slot per (CTA, split tile)
       // the CTA's segment of tile t is its first or its last segment
       const long long b = range_begin(cc, total, G), e = range_begin(cc + 1, total, G) - 1;

@@ -102,11 +102,20 @@ struct LinearShape {
   // slots): "ready" (the step's dequant group has written its TMEM slot and
   // seen its x stage land) and "freed" (the step's MMAs have completed).
   static constexpr int kL = lcm_int(kR, kRX);
-  // wfull, wempty [SW]; xfull [RX]; ready, freed [L]; dfull, dempty, done, epi[2]
-  static constexpr int kNumBars = 2 * kSW + kRX + 2 * kL + 5;
+  // wfull, wempty [SW]; xfull [RX]; ready, freed [L]; dfull, dempty, done
+  static constexpr int kNumBars = 2 * kSW + kRX + 2 * kL + 3;
   // columns per TMEM read in the epilogue: kIssuers reads of kEC 32-bit columns
   static constexpr int kEC = 32 / kIssuers;
-  static constexpr int kBarrierBytes = 1024;
+  // Split-tile fix-up at the end of a CTA's range, when every ring is idle:
+  // each epilogue warp owns kFixBufs buffers (2 KB: one contributor's 16
+  // partial columns of the warp's 32 rows) in the rings' space, each with a
+  // copy barrier after the kNumBars above.
+  static constexpr int kFixCols = 16;     // the shared-memory reads take 16 columns
+  static constexpr int kFixBlock = kFixCols * 32 * 4;
+  static constexpr int kFixBytes = kBarOff / 4 / kFixBlock * kFixBlock;
+  static constexpr int kFixBufs = (kFixBytes / kFixBlock < 16) ? kFixBytes / kFixBlock : 16;
+  static constexpr int kAllBars = kNumBars + 4 * kFixBufs;
+  static constexpr int kBarrierBytes = 2048;
   static constexpr int kSmemBytes = kBarOff + kBarrierBytes + 1024;  // + alignment slack
   static_assert(kXTile % 1024 == 0 && kTileBytes % 1024 == 0, "1024-byte aligned tiles");
   static_assert(kSW % kDeqGroups == 0 && kR % kDeqGroups == 0, "ring slots owned by one group");
@@ -115,8 +124,9 @@ struct LinearShape {
   // li - R, whose MMAs have completed.  So no parity wait can alias.
   static_assert(kRX % kDeqGroups == 0 || kRX >= kR, "x stage phases seen in order");
   static_assert(kDCol + kIssuers * NCOL <= static_cast<int>(kTmemCols), "TMEM budget");
-  static_assert(kNumBars * 8 + 32 <= kBarrierBytes, "barrier area");
-  static_assert(kNumBars <= kLinearThreads, "one thread per barrier at set-up");
+  static_assert(kFixBufs >= 2, "fix-up buffers");
+  static_assert(kAllBars * 8 + 32 <= kBarrierBytes, "barrier area");
+  static_assert(kAllBars <= kLinearThreads, "one thread per barrier at set-up");
   static_assert(kSmemBytes <= 232448, "shared memory");
 };
 
@@ -125,7 +135,7 @@ struct LinearParams {
   const uint8_t* packed;
   const uint16_t* scales;
   uint16_t* y;
-  float* partials;       // [2*G][NCOL][128] fp32
+  float* partials;       // [2*G][4][NCOL][32] fp32: slot, row quarter, column, row
   uint32_t* counters;    // [kMaxGrid], indexed by a split tile's first CTA; zero on entry and exit
   int M, N, K;
   int n_tiles, m_tiles, k_tiles;   // k_tiles = K / 64
@@ -143,11 +153,23 @@ __host__ __device__ __forceinline__ long long range_begin(int c, long long total
 __host__ __device__ __forceinline__ int range_owner(long long i, long long total, int G) {
   return static_cast<int>(((i + 1) * G + total - 1) / total - 1);
 }
+// First float of the partial of slot `slot` for row quarter q (32 rows):
+// NCOL columns of 32 consecutive floats, 128 * NCOL contiguous bytes.
+__host__ __device__ __forceinline__ long long partial_offset(int slot, int q, int ncol) {
+  return (static_cast<long long>(slot) * 4 + q) * ncol * 32;
+}
 // Partial slot of CTA c's segment in tile t (KS steps per tile): 0 for the
 // tile its range starts in, 1 for the tile its range ends in (only those two
 // can be partial).
 __host__ __device__ __forceinline__ int partial_slot(int c, long long t, long long total, int G, int KS) {
   return 2 * c + ((range_begin(c, total, G) / KS == t) ? 0 : 1);
+}
+// The same slot for contributor cc of split tile t (first contributor c_lo),
+// without divisions: t is the first tile of every contributor after c_lo,
+// and c_lo's first tile exactly when lo_first (its range starts at t's first
+// step).
+__host__ __device__ __forceinline__ int split_slot(int cc, int c_lo, bool lo_first) {
+  return cc == c_lo ? 2 * c_lo + (lo_first ? 0 : 1) : 2 * cc;
 }
 
 // Rows n of a warp's lanes, columns (tokens) m0 + j, j < C, of y as fp16
@@ -160,16 +182,31 @@ __device__ __forceinline__ void store_y_pairs(uint16_t* y, const float (&v)[C], 
                                               int N, int n, int lane) {
   static_assert(C % 2 == 0, "column pairs");
   const int odd = lane & 1;
-  uint32_t* yw = reinterpret_cast<uint32_t*>(y);
+  uint32_t* yw = reinterpret_cast<uint32_t*>(y) + (((m0 + odd) * N + (n - odd)) >> 1);
+  const long long step = N;                     // two tokens, in 32-bit words
+  // Eight pairs at a time: their conversions and exchanges first, then the
+  // stores, so no store waits on the latency of the next pair's shuffle.
+  constexpr int P = (C / 2 < 8) ? C / 2 : 8;
+  static_assert((C / 2) % P == 0, "pair groups");
 #pragma unroll
-  for (int j = 0; j < C; j += 2) {
-    const uint32_t ha = __half_as_ushort(__float2half_rn(v[j] * mul));
-    const uint32_t hb = __half_as_ushort(__float2half_rn(v[j + 1] * mul));
-    const uint32_t other = __shfl_xor_sync(0xffffffffu, odd ? ha : hb, 1);
-    const uint32_t lo = odd ? other : ha;       // row n - odd
-    const uint32_t hi = odd ? hb : other;       // row n - odd + 1
-    const int t = j + odd;
-    if (t < count) yw[((m0 + t) * N + (n - odd)) >> 1] = lo | (hi << 16);
+  for (int q0 = 0; q0 < C / 2; q0 += P) {
+    uint32_t keep[P], send[P];
+#pragma unroll
+    for (int q = 0; q < P; ++q) {
+      const uint32_t ha = __half_as_ushort(__float2half_rn(v[2 * (q0 + q)] * mul));
+      const uint32_t hb = __half_as_ushort(__float2half_rn(v[2 * (q0 + q) + 1] * mul));
+      keep[q] = odd ? hb : ha;
+      send[q] = odd ? ha : hb;
+    }
+#pragma unroll
+    for (int q = 0; q < P; ++q) send[q] = __shfl_xor_sync(0xffffffffu, send[q], 1);
+#pragma unroll
+    for (int q = 0; q < P; ++q) {
+      // even lane: (own, neighbour's) at token 2q, rows n, n+1; odd lane:
+      // (neighbour's, own) at token 2q+1, rows n-1, n
+      const uint32_t word = odd ? (send[q] | (keep[q] << 16)) : (keep[q] | (send[q] << 16));
+      if (2 * (q0 + q) + odd < count) yw[(q0 + q) * step] = word;
+    }
   }
 }
 
@@ -243,10 +280,9 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
   uint64_t* dfull = freed + kL;
   uint64_t* dempty = dfull + 1;
   uint64_t* done = dempty + 1;
-  uint64_t* epi = done + 1;                       // [2]: fix-up meeting of the first / last split segment
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + S::kNumBars);
-  volatile int* s_last = reinterpret_cast<volatile int*>(tmem_holder + 1);  // [2]
-  volatile int* s_abort = s_last + 2;
+  uint64_t* fixbar = done + 1;                    // [4][kFixBufs]: fix-up copies, per epilogue warp
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + S::kAllBars);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_holder + 1);
   volatile int* s_never = s_abort + 1;            // an abort flag nothing raises (final drains)
 
   const int warp = threadIdx.x >> 5;
@@ -268,7 +304,8 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
   grid_launch_dependents();
 
   // Barrier set-up, one thread per barrier.
-  if (threadIdx.x < S::kNumBars) {
+  static_assert(S::kIssuers == 1, "the general kernel runs 128 or 256 token columns");
+  if (threadIdx.x < S::kAllBars) {
     const int b = threadIdx.x;
     const int bx = 2 * kSW, br = bx + kRX, bf = br + kL, bd = bf + kL;
     uint32_t count = 1;                                       // wfull, xfull: producer arrive + tx
@@ -278,13 +315,11 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
     else if (b == bd) count = kISS;                           // dfull
     else if (b == bd + 1) count = 4;                          // dempty: epilogue warps
     else if (b == bd + 2) count = kISS;                       // done
-    else if (b >= bd + 3) count = 4;                          // epi[0], epi[1]
+    else if (b >= bd + 3) count = 1;                          // fix-up copies: lane 0 arrive + tx
     mbar_init(smem_u32(&bars[b]), count);
     fence_barrier_init();
   }
   if (threadIdx.x == 0) {
-    s_last[0] = 0;
-    s_last[1] = 0;
     *s_abort = 0;
     *s_never = 0;
   }
@@ -421,11 +456,27 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
     }
   } else if (warp >= kEpiWarp && warp < kEpiWarp + 4) {
     // ---------------- epilogue warpgroup: segments in order ----------------
+    // A split tile is finished without any wait on another CTA or warp.  Each
+    // epilogue warp (32 rows) counts on its own counter, p.counters[4*c_lo + q]:
+    //  - c_lo (the CTA holding the tile's first steps; for c_lo that is always
+    //    its last segment) finishes the tile at once if every later
+    //    contributor has counted; otherwise it publishes its partial and counts;
+    //  - a later contributor publishes its partial and counts;
+    //  - the one whose count completes the set (c_lo's and all later ones)
+    //    finishes the tile.
+    // Finishing sums the partials in CTA order c_lo .. c_hi, this CTA's own
+    // from TMEM when its accumulator still holds it (its last segment: no
+    // MMA follows), so y does not depend on which CTA finishes.  In the last
+    // segment every ring is idle and the other contributors' partials come in
+    // by bulk copies into that space, all in flight together; otherwise by
+    // loads, 32 columns of one contributor per round trip.
     grid_dependency_wait();                  // y, partials and counters may be in use before this kernel
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
-    const bool leader = (warp == kEpiWarp) && lane == 0;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t dacc = tmem + lane_base + S::kDCol;
+    const uint32_t mybar = smem_u32(fixbar) + quad * S::kFixBufs * 8;   // this warp's copy barriers
+    const uint32_t mybuf = smem_u32(smem) + quad * S::kFixBytes;        // and buffers
     int sg = 0;
     for (long long tile = tile_first; tile <= tile_last; ++tile, ++sg) {
       if (!warp_wait(smem_u32(dfull), sg & 1, s_abort)) break;
@@ -438,80 +489,145 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
       const float mul = __half2float(__ushort_as_half(p.scales[n]));
       const int c_lo = range_owner(tile * KS, total, G);
       const int c_hi = range_owner(tile * KS + KS - 1, total, G);
-      const bool split = c_lo != c_hi;
-      const int which = (tile == tile_first) ? 0 : 1;   // this CTA's first or last segment
-      float* part = p.partials + static_cast<long long>(2 * c + which) * NCOL * 128;
-      for (int c0 = 0; c0 < NCOL; c0 += kEC) {
-        // kEC columns of every issuer's accumulator, read together, summed
-        // in issuer order
-        uint32_t v[kISS][kEC];
-#pragma unroll
-        for (int i = 0; i < kISS; ++i) tmem_ld_cols<kEC>(tmem + lane_base + S::kDCol + i * NCOL + c0, v[i]);
+      const bool last_seg = tile == tile_last;
+
+      // 32 accumulator columns from c0 (this CTA's own sums for the segment).
+      auto own32 = [&](int c0, float (&a)[32]) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(dacc + c0, v);
         tmem_wait_ld();
-        float acc[kEC];
 #pragma unroll
-        for (int j = 0; j < kEC; ++j) {
-          float a = __uint_as_float(v[0][j]);
-#pragma unroll
-          for (int i = 1; i < kISS; ++i) a += __uint_as_float(v[i][j]);
-          acc[j] = a;
+        for (int j = 0; j < 32; ++j) a[j] = __uint_as_float(v[j]);
+      };
+      // The accumulator is read: the next segment's MMAs may overwrite it.
+      auto release_acc = [&]() {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(dempty));
+      };
+
+      if (c_lo == c_hi) {
+        for (int c0 = 0; c0 < NCOL; c0 += 32) {
+          float a[32];
+          own32(c0, a);
+          if (c0 + 32 >= NCOL) release_acc();
+          store_y_pairs<32>(p.y, a, mul, m0 + c0, mcount - c0, p.N, n, lane);
         }
-        if (c0 + kEC >= NCOL) {
-          // accumulators fully read: the next segment may overwrite them
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(dempty));
-        }
-        if (split) {
-#pragma unroll
-          for (int j = 0; j < kEC; ++j) __stcg(part + (c0 + j) * 128 + r, acc[j]);
-        } else {
-          store_y_pairs<kEC>(p.y, acc, mul, m0 + c0, mcount - c0, p.N, n, lane);
-        }
+        continue;
       }
-      if (split) {
-        // Publish this CTA's partial (release), count arrivals; the last CTA of
-        // the tile (acquire) sums every partial in CTA order.  The group's warps
-        // meet on an mbarrier (bounded wait), never on bar.sync, so an aborted
-        // warp cannot strand the others.  Each of the CTA's (at most two) split
-        // segments has its own meeting barrier.
-        const uint32_t eb = smem_u32(&epi[which]);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(eb);
-        if (!warp_wait(eb, 0, s_abort)) break;
-        if (leader) {
-          fence_acq_rel_gpu();
-          const unsigned int prev = atomicAdd(&p.counters[c_lo], 1u);
-          fence_acq_rel_gpu();
-          s_last[which] = (prev == static_cast<unsigned int>(c_hi - c_lo)) ? 1 : 0;
+
+      const unsigned int need = static_cast<unsigned int>(c_hi - c_lo);   // adds of the later contributors
+      unsigned int* cnt = p.counters + 4 * c_lo + quad;
+      const bool lo_first = range_begin(c_lo, total, G) == tile * KS;
+      auto part_of = [&](int cc) -> const float* {
+        return p.partials + partial_offset(split_slot(cc, c_lo, lo_first), quad, NCOL);
+      };
+      bool finish;
+      if (c == c_lo && __all_sync(0xffffffffu, ld_acquire(cnt) == need)) {
+        finish = true;                       // every later partial is there
+      } else {
+        // Publish this CTA's partial, then count (release).  The lanes' stores
+        // are ordered before lane 0's add by the warp barrier, and its release
+        // publishes them with its own.
+        float* mine = p.partials + partial_offset(2 * c + ((tile == tile_first) ? 0 : 1), quad, NCOL) + lane;
+        for (int c0 = 0; c0 < NCOL; c0 += 16) {
+          uint32_t v[16];
+          tmem_ld_32x32b_x16(dacc + c0, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) __stcg(mine + (c0 + j) * 32, __uint_as_float(v[j]));
+        }
+        release_acc();
+        unsigned int old = 0;
+        if (lane == 0) old = atom_add_acq_rel(cnt, 1u);
+        finish = __shfl_sync(0xffffffffu, old, 0) == need;
+        if (finish) (void)ld_acquire(cnt);   // every lane acquires the others' partials
+      }
+      if (!finish) continue;
+
+      bool ok = true;
+      if (last_seg) {
+        // Own sums from TMEM; the other nm contributors' kFixCols-column
+        // blocks (item k: block k / nm, k-th other contributor k % nm)
+        // through the warp's kFixBufs copy buffers.
+        constexpr int FC = S::kFixCols;
+        const int nm = c_hi - c_lo;
+        const int nblk = (mcount + FC - 1) / FC;
+        const int items = nblk * nm;
+        auto issue = [&](int k) {            // lane 0
+          const int o = k % nm;
+          const int cc = c_lo + o + ((c_lo + o >= c) ? 1 : 0);
+          const int b = k % S::kFixBufs;
+          const uint32_t bar = mybar + b * 8;
+          mbar_arrive_expect_tx(bar, static_cast<uint32_t>(S::kFixBlock));
+          bulk_load(mybuf + b * S::kFixBlock, part_of(cc) + (k / nm) * FC * 32,
+                    static_cast<uint32_t>(S::kFixBlock), bar, policy_evict_first());
+        };
+        int issued = min(items, S::kFixBufs);
+        if (lane == 0) {
+          fence_proxy_async_all();           // the acquired partials, for the copies
+          for (int k = 0; k < issued; ++k) issue(k);
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(eb);
-        if (!warp_wait(eb, 1, s_abort)) break;
-        if (s_last[which]) {
-          // kSumCols columns of one contributor per step: their loads are all
-          // in flight together, so a tile costs about (NCOL / kSumCols) x
-          // contributors L2 round trips rather than one per 8 columns.
-          constexpr int kSumCols = NCOL < 32 ? NCOL : 32;
-          for (int c0 = 0; c0 < mcount; c0 += kSumCols) {
-            float acc[kSumCols];
+        int k = 0;
+        for (int blk = 0; blk < nblk && ok; ++blk) {
+          float acc[FC];
 #pragma unroll
-            for (int j = 0; j < kSumCols; ++j) acc[j] = 0.0f;
-            for (int cc = c_lo; cc <= c_hi; ++cc) {
-              const float* src = p.partials +
-                                 static_cast<long long>(partial_slot(cc, tile, total, G, KS)) * NCOL * 128 +
-                                 c0 * 128 + r;
-              float v[kSumCols];
+          for (int j = 0; j < FC; ++j) acc[j] = 0.0f;
+          for (int cc = c_lo; cc <= c_hi; ++cc) {
+            if (cc == c) {
+              uint32_t v[FC];
+              tmem_ld_cols<FC>(dacc + blk * FC, v);
+              tmem_wait_ld();
 #pragma unroll
-              for (int j = 0; j < kSumCols; ++j) v[j] = __ldcg(src + j * 128);
-#pragma unroll
-              for (int j = 0; j < kSumCols; ++j) acc[j] += v[j];
+              for (int j = 0; j < FC; ++j) acc[j] += __uint_as_float(v[j]);
+              continue;
             }
-            store_y_pairs<kSumCols>(p.y, acc, mul, m0 + c0, mcount - c0, p.N, n, lane);
+            const int b = k % S::kFixBufs;
+            if (!warp_wait(mybar + b * 8, (k / S::kFixBufs) & 1, s_abort)) {
+              ok = false;
+              break;
+            }
+            float v[FC];
+            ld_shared_f32x16_stride128(mybuf + b * S::kFixBlock + lane * 4, v);
+#pragma unroll
+            for (int j = 0; j < FC; ++j) acc[j] += v[j];
+            __syncwarp();                    // every lane has read the buffer
+            if (k + S::kFixBufs < items) {
+              if (lane == 0) {
+                fence_proxy_async_smem();
+                issue(k + S::kFixBufs);
+              }
+              ++issued;
+            }
+            ++k;
           }
-          if (leader) p.counters[c_lo] = 0u;
+          if (ok) store_y_pairs<FC>(p.y, acc, mul, m0 + blk * FC, mcount - blk * FC, p.N, n, lane);
+        }
+        // Leave no copy in flight.
+        for (; k < issued; ++k) warp_wait(mybar + (k % S::kFixBufs) * 8, (k / S::kFixBufs) & 1, s_never);
+      } else {
+        // Every partial from memory (this CTA's too: its accumulator may
+        // already hold the next segment's sums), 16 columns of one
+        // contributor per round trip.
+        for (int c0 = 0; c0 < mcount; c0 += 16) {
+          float acc[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) acc[j] = 0.0f;
+          for (int cc = c_lo; cc <= c_hi; ++cc) {
+            const float* src = part_of(cc) + c0 * 32 + lane;
+            float v[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] = __ldcg(src + j * 32);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) acc[j] += v[j];
+          }
+          store_y_pairs<16>(p.y, acc, mul, m0 + c0, mcount - c0, p.N, n, lane);
         }
       }
+      if (!ok) break;
+      __syncwarp();
+      if (lane == 0) *cnt = 0u;              // every contributor has counted: reset for the next launch
     }
   }
 

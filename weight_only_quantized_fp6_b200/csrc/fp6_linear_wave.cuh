@@ -92,8 +92,8 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
 
   grid_launch_dependents();
 
-  // Barrier set-up as in the general kernel (its split-K meeting barriers
-  // stay unused here).
+  // Barrier set-up as in the general kernel (without its split-tile copy
+  // barriers).
   if (threadIdx.x < S::kNumBars) {
     const int b = threadIdx.x;
     const int bx = 2 * kSW, br = bx + kRX, bf = br + kL, bd = bf + kL;
@@ -104,7 +104,6 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
     else if (b == bd) count = kISS;                           // dfull
     else if (b == bd + 1) count = 4;                          // dempty: epilogue warps
     else if (b == bd + 2) count = kISS;                       // done
-    else if (b >= bd + 3) count = 4;
     mbar_init(smem_u32(&bars[b]), count);
     fence_barrier_init();
   }

@@ -29,6 +29,28 @@ __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
 __device__ __forceinline__ void fence_barrier_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
+// 16 floats at addr + 128 * j (j = 0..15) from shared memory, issued back to
+// back (one statement, so no use of an earlier one stalls the later loads).
+__device__ __forceinline__ void ld_shared_f32x16_stride128(uint32_t addr, float (&v)[16]) {
+  asm volatile(
+      "ld.shared.f32 %0, [%16];\n\tld.shared.f32 %1, [%16+128];\n\t"
+      "ld.shared.f32 %2, [%16+256];\n\tld.shared.f32 %3, [%16+384];\n\t"
+      "ld.shared.f32 %4, [%16+512];\n\tld.shared.f32 %5, [%16+640];\n\t"
+      "ld.shared.f32 %6, [%16+768];\n\tld.shared.f32 %7, [%16+896];\n\t"
+      "ld.shared.f32 %8, [%16+1024];\n\tld.shared.f32 %9, [%16+1152];\n\t"
+      "ld.shared.f32 %10, [%16+1280];\n\tld.shared.f32 %11, [%16+1408];\n\t"
+      "ld.shared.f32 %12, [%16+1536];\n\tld.shared.f32 %13, [%16+1664];\n\t"
+      "ld.shared.f32 %14, [%16+1792];\n\tld.shared.f32 %15, [%16+1920];"
+      : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7]),
+        "=f"(v[8]), "=f"(v[9]), "=f"(v[10]), "=f"(v[11]), "=f"(v[12]), "=f"(v[13]), "=f"(v[14]), "=f"(v[15])
+      : "r"(addr)
+      : "memory");
+}
+// Orders this thread's earlier generic-proxy accesses (and those it has
+// acquired) before its later async-proxy (bulk copy) accesses, all state spaces.
+__device__ __forceinline__ void fence_proxy_async_all() {
+  asm volatile("fence.proxy.async;" ::: "memory");
+}
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
