@@ -107,14 +107,16 @@ struct LinearShape {
   // columns per TMEM read in the epilogue: kIssuers reads of kEC 32-bit columns
   static constexpr int kEC = 32 / kIssuers;
   // Split-tile fix-up at the end of a CTA's range, when every ring is idle:
-  // each epilogue warp owns kFixBufs buffers (2 KB: one contributor's 16
-  // partial columns of the warp's 32 rows) in the rings' space, each with a
-  // copy barrier after the kNumBars above.
+  // the epilogue warp and the three dequant warps of each row quarter (16
+  // warps) each own kFixBufs buffers (2 KB: one contributor's 16 partial
+  // columns of the quarter's 32 rows) in the rings' space, each with a copy
+  // barrier after the kNumBars above; then one "go" barrier per quarter.
   static constexpr int kFixCols = 16;     // the shared-memory reads take 16 columns
   static constexpr int kFixBlock = kFixCols * 32 * 4;
-  static constexpr int kFixBytes = kBarOff / 4 / kFixBlock * kFixBlock;
+  static constexpr int kFixWarps = 4 * (1 + kDeqGroups);
+  static constexpr int kFixBytes = kBarOff / kFixWarps / kFixBlock * kFixBlock;
   static constexpr int kFixBufs = (kFixBytes / kFixBlock < 16) ? kFixBytes / kFixBlock : 16;
-  static constexpr int kAllBars = kNumBars + 4 * kFixBufs;
+  static constexpr int kAllBars = kNumBars + kFixWarps * kFixBufs + 4;
   static constexpr int kBarrierBytes = 2048;
   static constexpr int kSmemBytes = kBarOff + kBarrierBytes + 1024;  // + alignment slack
   static_assert(kXTile % 1024 == 0 && kTileBytes % 1024 == 0, "1024-byte aligned tiles");
@@ -258,6 +260,77 @@ __device__ __forceinline__ void fence_acq_rel_gpu() {
   asm volatile("fence.acq_rel.gpu;" ::: "memory");
 }
 
+// Finishes column blocks rank, rank + 4, ... (kFixCols columns each, below
+// mcount) of a split tile, for the 32 rows of one row quarter, at the end of
+// the CTA's range (every ring idle, this CTA's accumulator final): its own
+// sums come from TMEM (dacc), the other contributors' partials by bulk copies
+// into this warp's kFixBufs buffers (shared addresses buf, barriers bar), all
+// summed in CTA order c_lo .. c_hi, then scaled and stored.  False if a wait
+// gave up.
+template <int NCOL, class S>
+__device__ __forceinline__ bool finish_blocks(const LinearParams& p, int c, int c_lo, int c_hi, bool lo_first, int quad,
+                                              int lane, int rank, uint32_t dacc, uint32_t bar, uint32_t buf, int m0,
+                                              int mcount, int n, float mul, volatile int* abort, volatile int* never) {
+  constexpr int FC = S::kFixCols;
+  const int nm = c_hi - c_lo;                        // contributors read from memory
+  const int nblk_all = (mcount + FC - 1) / FC;
+  const int nblk = rank < nblk_all ? (nblk_all - rank + 3) / 4 : 0;
+  const int items = nblk * nm;                       // item k: this warp's block k / nm, other k % nm
+  auto issue = [&](int k) {                          // lane 0
+    const int o = k % nm;
+    const int cc = c_lo + o + ((c_lo + o >= c) ? 1 : 0);
+    const int blk = rank + 4 * (k / nm);
+    const int b = k % S::kFixBufs;
+    mbar_arrive_expect_tx(bar + b * 8, static_cast<uint32_t>(S::kFixBlock));
+    bulk_load(buf + b * S::kFixBlock,
+              p.partials + partial_offset(split_slot(cc, c_lo, lo_first), quad, NCOL) + blk * FC * 32,
+              static_cast<uint32_t>(S::kFixBlock), bar + b * 8, policy_evict_first());
+  };
+  int issued = min(items, S::kFixBufs);
+  if (lane == 0) {
+    fence_proxy_async_all();                         // the acquired partials, for the copies
+    for (int k = 0; k < issued; ++k) issue(k);
+  }
+  __syncwarp();
+  int k = 0;
+  bool ok = true;
+  for (int kb = 0; kb < nblk && ok; ++kb) {
+    const int blk = rank + 4 * kb;
+    float acc[FC];
+#pragma unroll
+    for (int j = 0; j < FC; ++j) acc[j] = 0.0f;
+    for (int cc = c_lo; cc <= c_hi; ++cc) {
+      if (cc == c) {
+        uint32_t v[FC];
+        tmem_ld_cols<FC>(dacc + blk * FC, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < FC; ++j) acc[j] += __uint_as_float(v[j]);
+        continue;
+      }
+      const int b = k % S::kFixBufs;
+      if (!warp_wait(bar + b * 8, (k / S::kFixBufs) & 1, abort)) {
+        ok = false;
+        break;
+      }
+      float v[FC];
+      ld_shared_f32x16_stride128(buf + b * S::kFixBlock + lane * 4, v);
+#pragma unroll
+      for (int j = 0; j < FC; ++j) acc[j] += v[j];
+      __syncwarp();                                  // every lane has read the buffer: refill it
+      if (k + S::kFixBufs < items) {
+        if (lane == 0) issue(k + S::kFixBufs);
+        ++issued;
+      }
+      ++k;
+    }
+    if (ok) store_y_pairs<FC>(p.y, acc, mul, m0 + blk * FC, mcount - blk * FC, p.N, n, lane);
+  }
+  // Leave no copy in flight.
+  for (; k < issued; ++k) warp_wait(bar + (k % S::kFixBufs) * 8, (k / S::kFixBufs) & 1, never);
+  return ok;
+}
+
 template <int NCOL, Fmt F = Fmt::E3M2>
 __global__ void __launch_bounds__(kLinearThreads, 1)
     fp6_linear_kernel(const __grid_constant__ CUtensorMap tmap_x, const LinearParams p) {
@@ -280,10 +353,12 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
   uint64_t* dfull = freed + kL;
   uint64_t* dempty = dfull + 1;
   uint64_t* done = dempty + 1;
-  uint64_t* fixbar = done + 1;                    // [4][kFixBufs]: fix-up copies, per epilogue warp
+  uint64_t* fixbar = done + 1;                    // [16][kFixBufs]: fix-up copies, per warp (quarter, rank)
+  uint64_t* fixgo = fixbar + S::kFixWarps * S::kFixBufs;   // [4]: a quarter's fix-up posted
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + S::kAllBars);
   volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_holder + 1);
   volatile int* s_never = s_abort + 1;            // an abort flag nothing raises (final drains)
+  volatile int* s_fixgo = s_never + 1;            // [4]: 1 if the quarter's last tile is finished here
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -315,7 +390,7 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
     else if (b == bd) count = kISS;                           // dfull
     else if (b == bd + 1) count = 4;                          // dempty: epilogue warps
     else if (b == bd + 2) count = kISS;                       // done
-    else if (b >= bd + 3) count = 1;                          // fix-up copies: lane 0 arrive + tx
+    else if (b >= bd + 3) count = 1;                          // fix-up copies (arrive + tx), go
     mbar_init(smem_u32(&bars[b]), count);
     fence_barrier_init();
   }
@@ -454,6 +529,22 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&ready[li % kL]));
     }
+    // The end of the range: help finish the CTA's last tile if the epilogue
+    // warp of this row quarter finishes it (blocks 1 + g, 5 + g, ...).
+    if (warp_wait(smem_u32(&fixgo[quad]), 0, s_abort) && s_fixgo[quad]) {
+      tc_fence_after();
+      const long long tile = tile_last;
+      const int nt = static_cast<int>(tile / MT);
+      const int mt = static_cast<int>(tile - static_cast<long long>(nt) * MT);
+      const int n = nt * kTileRows + r;
+      const int c_lo = range_owner(tile * KS, total, G);
+      const int rank = 1 + g;
+      finish_blocks<NCOL, S>(p, c, c_lo, range_owner(tile * KS + KS - 1, total, G),
+                             range_begin(c_lo, total, G) == tile * KS, quad, lane, rank,
+                             tmem + lane_base + S::kDCol, smem_u32(fixbar) + (quad * 4 + rank) * S::kFixBufs * 8,
+                             smem_u32(smem) + (quad * 4 + rank) * S::kFixBytes, mt * NCOL, min(NCOL, p.M - mt * NCOL),
+                             n, __half2float(__ushort_as_half(p.scales[n])), s_abort, s_never);
+    }
   } else if (warp >= kEpiWarp && warp < kEpiWarp + 4) {
     // ---------------- epilogue warpgroup: segments in order ----------------
     // A split tile is finished without any wait on another CTA or warp.  Each
@@ -475,8 +566,7 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
     const int r = quad * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t dacc = tmem + lane_base + S::kDCol;
-    const uint32_t mybar = smem_u32(fixbar) + quad * S::kFixBufs * 8;   // this warp's copy barriers
-    const uint32_t mybuf = smem_u32(smem) + quad * S::kFixBytes;        // and buffers
+    bool posted = false;                     // the quarter's dequant warps have been told
     int sg = 0;
     for (long long tile = tile_first; tile <= tile_last; ++tile, ++sg) {
       if (!warp_wait(smem_u32(dfull), sg & 1, s_abort)) break;
@@ -547,65 +637,16 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
 
       bool ok = true;
       if (last_seg) {
-        // Own sums from TMEM; the other nm contributors' kFixCols-column
-        // blocks (item k: block k / nm, k-th other contributor k % nm)
-        // through the warp's kFixBufs copy buffers.
-        constexpr int FC = S::kFixCols;
-        const int nm = c_hi - c_lo;
-        const int nblk = (mcount + FC - 1) / FC;
-        const int items = nblk * nm;
-        auto issue = [&](int k) {            // lane 0
-          const int o = k % nm;
-          const int cc = c_lo + o + ((c_lo + o >= c) ? 1 : 0);
-          const int b = k % S::kFixBufs;
-          const uint32_t bar = mybar + b * 8;
-          mbar_arrive_expect_tx(bar, static_cast<uint32_t>(S::kFixBlock));
-          bulk_load(mybuf + b * S::kFixBlock, part_of(cc) + (k / nm) * FC * 32,
-                    static_cast<uint32_t>(S::kFixBlock), bar, policy_evict_first());
-        };
-        int issued = min(items, S::kFixBufs);
+        // Post the tile to the quarter's dequant warps (no MMA or ring use
+        // follows), then take this warp's share: blocks 0, 4, 8, ...
         if (lane == 0) {
-          fence_proxy_async_all();           // the acquired partials, for the copies
-          for (int k = 0; k < issued; ++k) issue(k);
+          s_fixgo[quad] = 1;
+          mbar_arrive(smem_u32(&fixgo[quad]));
         }
-        __syncwarp();
-        int k = 0;
-        for (int blk = 0; blk < nblk && ok; ++blk) {
-          float acc[FC];
-#pragma unroll
-          for (int j = 0; j < FC; ++j) acc[j] = 0.0f;
-          for (int cc = c_lo; cc <= c_hi; ++cc) {
-            if (cc == c) {
-              uint32_t v[FC];
-              tmem_ld_cols<FC>(dacc + blk * FC, v);
-              tmem_wait_ld();
-#pragma unroll
-              for (int j = 0; j < FC; ++j) acc[j] += __uint_as_float(v[j]);
-              continue;
-            }
-            const int b = k % S::kFixBufs;
-            if (!warp_wait(mybar + b * 8, (k / S::kFixBufs) & 1, s_abort)) {
-              ok = false;
-              break;
-            }
-            float v[FC];
-            ld_shared_f32x16_stride128(mybuf + b * S::kFixBlock + lane * 4, v);
-#pragma unroll
-            for (int j = 0; j < FC; ++j) acc[j] += v[j];
-            __syncwarp();                    // every lane has read the buffer
-            if (k + S::kFixBufs < items) {
-              if (lane == 0) {
-                fence_proxy_async_smem();
-                issue(k + S::kFixBufs);
-              }
-              ++issued;
-            }
-            ++k;
-          }
-          if (ok) store_y_pairs<FC>(p.y, acc, mul, m0 + blk * FC, mcount - blk * FC, p.N, n, lane);
-        }
-        // Leave no copy in flight.
-        for (; k < issued; ++k) warp_wait(mybar + (k % S::kFixBufs) * 8, (k / S::kFixBufs) & 1, s_never);
+        posted = true;
+        ok = finish_blocks<NCOL, S>(p, c, c_lo, c_hi, lo_first, quad, lane, 0, dacc,
+                                    smem_u32(fixbar) + quad * 4 * S::kFixBufs * 8,
+                                    smem_u32(smem) + quad * 4 * S::kFixBytes, m0, mcount, n, mul, s_abort, s_never);
       } else {
         // Every partial from memory (this CTA's too: its accumulator may
         // already hold the next segment's sums), 16 columns of one
@@ -628,6 +669,10 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
       if (!ok) break;
       __syncwarp();
       if (lane == 0) *cnt = 0u;              // every contributor has counted: reset for the next launch
+    }
+    if (!posted && lane == 0) {              // nothing for the dequant warps to help with
+      s_fixgo[quad] = 0;
+      mbar_arrive(smem_u32(&fixgo[quad]));
     }
   }
 
