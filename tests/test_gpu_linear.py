@@ -75,6 +75,24 @@ def test_grid_shapes(fp6, orc, N, K):
         run_case(fp6, orc, N, K, M, N + K, M)
 
 
+@pytest.mark.parametrize("M,N,K", [(128, 128, 1024), (100, 256, 4096), (300, 128, 8192), (128, 128, 18944),
+                                   (65, 384, 8192)])
+def test_general_kernel_many_contributors(fp6, orc, M, N, K):
+    """The M > 64 kernel with row tiles split over 8 to 148 CTAs: the finish
+    at the end of a range draws more partials than a warp has copy buffers,
+    CTAs hold a first and a last segment of different tiles, and some tiles
+    are finished by a CTA that still has work.  Every output is compared, and
+    a second launch must give the same bits (the sum order does not depend
+    on which CTA finishes)."""
+    from weight_only_quantized_fp6_b200 import inputs
+    y, _ = run_case(fp6, orc, N, K, M, 9000 + N + K, 9100 + M)
+    W = inputs.weights(9000 + N + K, N, K)
+    x = inputs.activations(9100 + M, M, K)
+    codes, scales, packed = gpu_layer(fp6, W)
+    for _ in range(2):
+        assert np.array_equal(bits16(fp6.linear(as_f16(x), packed, scales, N, K)), y)
+
+
 def test_one_hot_bit_exact(fp6, orc):
     """x = identity rows: y[m,n] = fp16_rne(scale[n] * decode(c[n,m])) exactly."""
     from weight_only_quantized_fp6_b200 import inputs

@@ -88,7 +88,18 @@ struct LinearShape {
   static constexpr int kXStage = kTMax * kXTile;
   static constexpr int kTileBytes = Format<F>::kTileBytes;
   static constexpr int kWStage = kTMax * kTileBytes;
-  static constexpr int kIssuers = (NCOL <= 32) ? 4 : (NCOL == 64) ? 2 : 1;
+  // MMA-issuing warps.  Up to 64 token columns each takes a k-slice of every
+  // tile into its own accumulator (summed in the epilogue).  At 256 columns
+  // two issuers split the tokens instead (N = 128 each, every k-slice, one
+  // accumulator in two column halves): one thread issues an MMA in about
+  // 100 cycles, so a second issuing thread is what lets the tensor pipe run
+  // at its rate.
+  static constexpr int kIssuers = (NCOL <= 32) ? 4 : (NCOL == 64) ? 2 : (NCOL == 256) ? 2 : 1;
+  static constexpr bool kNSplit = NCOL == 256;
+  static constexpr int kIssN = kNSplit ? NCOL / kIssuers : NCOL;        // MMA N of one issuer
+  static constexpr int kIssSlices = kNSplit ? 4 : 4 / kIssuers;         // k-slices per tile and issuer
+  static constexpr int kAccIssuers = kNSplit ? 1 : kIssuers;            // accumulators the epilogue sums
+  static constexpr int kAccCols = kNSplit ? NCOL : kIssuers * NCOL;
   static constexpr int kRX = (NCOL == 16) ? 8 : (NCOL == 32) ? 4 : 3;     // x stages (>= 3)
   // weight stages of 6-bit tiles; the same bytes in FP4 tiles
   static constexpr int kSW = ((NCOL <= 32) ? 6 : (NCOL == 64) ? 12 : (NCOL == 128) ? 9 : 18) * 6144 / kTileBytes /
@@ -104,8 +115,8 @@ struct LinearShape {
   static constexpr int kL = lcm_int(kR, kRX);
   // wfull, wempty [SW]; xfull [RX]; ready, freed [L]; dfull, dempty, done
   static constexpr int kNumBars = 2 * kSW + kRX + 2 * kL + 3;
-  // columns per TMEM read in the epilogue: kIssuers reads of kEC 32-bit columns
-  static constexpr int kEC = 32 / kIssuers;
+  // columns per TMEM read in the epilogue: kAccIssuers reads of kEC 32-bit columns
+  static constexpr int kEC = 32 / kAccIssuers;
   // Split-tile fix-up at the end of a CTA's range, when every ring is idle:
   // the epilogue warp and the three dequant warps of each row quarter (16
   // warps) each own kFixBufs buffers (2 KB: one contributor's 16 partial
@@ -125,7 +136,7 @@ struct LinearShape {
   // fill (step li - RX) complete: it was its own step, or it precedes step
   // li - R, whose MMAs have completed.  So no parity wait can alias.
   static_assert(kRX % kDeqGroups == 0 || kRX >= kR, "x stage phases seen in order");
-  static_assert(kDCol + kIssuers * NCOL <= static_cast<int>(kTmemCols), "TMEM budget");
+  static_assert(kDCol + kAccCols <= static_cast<int>(kTmemCols), "TMEM budget");
   static_assert(kFixBufs >= 2, "fix-up buffers");
   static_assert(kAllBars * 8 + 32 <= kBarrierBytes, "barrier area");
   static_assert(kAllBars <= kLinearThreads, "one thread per barrier at set-up");
@@ -379,7 +390,7 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
   grid_launch_dependents();
 
   // Barrier set-up, one thread per barrier.
-  static_assert(S::kIssuers == 1, "the general kernel runs 128 or 256 token columns");
+  static_assert(S::kAccIssuers == 1, "the general kernel runs 128 or 256 token columns (one accumulator)");
   if (threadIdx.x < S::kAllBars) {
     const int b = threadIdx.x;
     const int bx = 2 * kSW, br = bx + kRX, bf = br + kL, bd = bf + kL;
@@ -456,11 +467,12 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
     for (int li = issued > kRX ? issued - kRX : 0; li < issued; ++li)
       warp_wait(smem_u32(&xfull[li % kRX]), (li / kRX) & 1, s_never);
   } else if (warp < kISS) {
-    // ---------------- MMA issuer `warp`: k-slice [warp*4/kISS, (warp+1)*4/kISS) of every tile ----------------
-    constexpr uint32_t idesc = idesc_f16_f32(128, NCOL);
-    constexpr int kSlice = 4 / kISS;
-    const int kk0 = warp * kSlice;
-    const uint32_t d_tmem = tmem + S::kDCol + warp * NCOL;
+    // ---------------- MMA issuer `warp`: its k-slices or its token half of every tile ----------------
+    constexpr uint32_t idesc = idesc_f16_f32(128, S::kIssN);
+    constexpr int kSlice = S::kIssSlices;
+    const int kk0 = S::kNSplit ? 0 : warp * kSlice;
+    const uint32_t d_tmem = tmem + S::kDCol + warp * (S::kNSplit ? S::kIssN : NCOL);
+    const uint32_t b_off = S::kNSplit ? warp * S::kIssN * 128 : 0;   // its tokens' rows of the x tile
     // The loop runs in lane 0 alone: a barrier test by one lane costs about
     // 13 cycles against about 110 for a whole warp, and a warp issues
     // tcgen05.mma at one per ~50 cycles whichever lanes issue, so per-step
@@ -477,7 +489,7 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
         if (!wait_bounded(smem_u32(&ready[li % kL]), (li / kL) & 1, s_abort)) break;
         {
           tc_fence_after();
-          const uint64_t bdesc0 = smem_desc_sw128(smem_u32(smem + sx * S::kXStage));
+          const uint64_t bdesc0 = smem_desc_sw128(smem_u32(smem + sx * S::kXStage) + b_off);
           const uint32_t a0 = tmem + s * S::kSlotCols;
           for (int t = 0; t < T; ++t) {
             // B descriptor of tile t: start address advances by kXTile bytes (>> 4)

@@ -166,11 +166,12 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
     for (int li = issued > kRX ? issued - kRX : 0; li < issued; ++li)
       warp_wait(smem_u32(&xfull[li % kRX]), (li / kRX) & 1, s_never);
   } else if (warp < kISS) {
-    // ---------------- MMA issuer `warp`: k-slice [warp*4/kISS, (warp+1)*4/kISS) of every tile ----------------
-    constexpr uint32_t idesc = idesc_f16_f32(128, NCOL);
-    constexpr int kSlice = 4 / kISS;
-    const int kk0 = warp * kSlice;
-    const uint32_t d_tmem = tmem + S::kDCol + warp * NCOL;
+    // ---------------- MMA issuer `warp`: its k-slices or its token half of every tile ----------------
+    constexpr uint32_t idesc = idesc_f16_f32(128, S::kIssN);
+    constexpr int kSlice = S::kIssSlices;
+    const int kk0 = S::kNSplit ? 0 : warp * kSlice;
+    const uint32_t d_tmem = tmem + S::kDCol + warp * (S::kNSplit ? S::kIssN : NCOL);
+    const uint32_t b_off = S::kNSplit ? warp * S::kIssN * 128 : 0;   // its tokens' rows of the x tile
     // The loop runs in lane 0 alone: a barrier test by one lane costs about
     // 13 cycles against about 110 for a whole warp, and a warp issues
     // tcgen05.mma at one per ~50 cycles whichever lanes issue, so per-step
@@ -187,7 +188,7 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
         if (!wait_bounded(smem_u32(&ready[li % kL]), (li / kL) & 1, s_abort)) break;
         {
           tc_fence_after();
-          const uint64_t bdesc0 = smem_desc_sw128(smem_u32(smem + sx * S::kXStage));
+          const uint64_t bdesc0 = smem_desc_sw128(smem_u32(smem + sx * S::kXStage) + b_off);
           const uint32_t a0 = tmem + s * S::kSlotCols;
           for (int t = 0; t < T; ++t) {
             const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(t * (S::kXTile >> 4));
@@ -254,16 +255,17 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
       const int mcount = min(NCOL, p.M - m0);
       const float mul = __half2float(__ushort_as_half(p.scales[n]));
       for (int c0 = 0; c0 < NCOL; c0 += kEC) {
-        uint32_t v[kISS][kEC];
+        constexpr int kAcc = S::kAccIssuers;
+        uint32_t v[kAcc][kEC];
 #pragma unroll
-        for (int i = 0; i < kISS; ++i) tmem_ld_cols<kEC>(tmem + lane_base + S::kDCol + i * NCOL + c0, v[i]);
+        for (int i = 0; i < kAcc; ++i) tmem_ld_cols<kEC>(tmem + lane_base + S::kDCol + i * NCOL + c0, v[i]);
         tmem_wait_ld();
         float acc[kEC];
 #pragma unroll
         for (int j = 0; j < kEC; ++j) {
           float a = __uint_as_float(v[0][j]);
 #pragma unroll
-          for (int i = 1; i < kISS; ++i) a += __uint_as_float(v[i][j]);
+          for (int i = 1; i < kAcc; ++i) a += __uint_as_float(v[i][j]);
           acc[j] = a;
         }
         if (c0 + kEC >= NCOL) {
