@@ -19,13 +19,14 @@
 //                 owns one weight row (its TMEM lane), reads its 48 packed bytes
 //                 per tile, rebuilds 64 fp16 weights (decode(c), exact) and stores
 //                 them into the step's TMEM slot (tcgen05.st);
-//   warps 0..3    MMA issuers: NISS warps each take a k-slice of every tile
-//                 (tcgen05.mma M = 128, N = NCOL, K = 16; A from the TMEM slot,
-//                 B = x from smem) into their own fp32 accumulator in TMEM;
+//   warps 0..3    MMA issuers (tcgen05.mma M = 128, K = 16; A from the TMEM
+//                 slot, B = x from smem): one for 128 token columns (N = 128),
+//                 two for 256, each issuing the MMAs of its 128 tokens into
+//                 its half of the fp32 accumulator in TMEM;
 //   warps 4..7    the epilogue warpgroup: per segment (the steps of one tile
-//                 that this CTA owns), tcgen05.ld of the NISS accumulators,
-//                 summed in a fixed order, * scale, fp16 store, or the
-//                 split-K partial and fix-up.
+//                 that this CTA owns), tcgen05.ld of the accumulator, * scale,
+//                 fp16 store, or the split-K partial and fix-up (with the
+//                 dequant warps' help at the end of the range).
 //
 // Rings: packed weights (SW smem stages, filled by the weight producer,
 // released by the dequant group), x (RX smem stages) and dequantized weights
@@ -352,7 +353,6 @@ __global__ void __launch_bounds__(kLinearThreads, 1)
   constexpr int kSW = S::kSW;
   constexpr int kISS = S::kIssuers;
   constexpr int kL = S::kL;
-  constexpr int kEC = S::kEC;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBarOff);
