@@ -470,39 +470,66 @@ def run_fp6(args, world, rank, local):
     # End to end through the public API with host buffers: every step copies
     # its five activation matrices host -> device from one pinned staging
     # buffer, runs the five layer calls (FP6Linear.__call__) and copies their
-    # five outputs device -> host into one pinned buffer.
+    # five outputs device -> host into a pinned buffer.  As a serving loop
+    # would, consecutive steps overlap: two sets of device buffers, the input
+    # copies on one copy stream and the output copies on another, so step
+    # s + 1's inputs travel while step s computes and step s's outputs while
+    # step s + 1 computes.  Every step's copies are inside the timed region.
     rows = sum(MS)
     x_host = torch.empty((rows, K_DIM), dtype=torch.float16).pin_memory()
-    y_host = torch.empty((rows, N_DIM), dtype=torch.float16).pin_memory()
+    y_host = [torch.empty((rows, N_DIM), dtype=torch.float16).pin_memory() for _ in range(2)]
     off = np.cumsum([0] + MS)
     for M, o in zip(MS, off):
         x_host[o:o + M].copy_(xs[M].cpu())
-    x_dev = torch.empty((rows, K_DIM), dtype=torch.float16, device=dev)
-    y_dev = torch.empty((rows, N_DIM), dtype=torch.float16, device=dev)
-    x_views = [x_dev[o:o + M] for M, o in zip(MS, off)]
-    y_views = [y_dev[o:o + M] for M, o in zip(MS, off)]
+    x_dev = [torch.empty((rows, K_DIM), dtype=torch.float16, device=dev) for _ in range(2)]
+    y_dev = [torch.empty((rows, N_DIM), dtype=torch.float16, device=dev) for _ in range(2)]
+    x_views = [[xd[o:o + M] for M, o in zip(MS, off)] for xd in x_dev]
+    y_views = [[yd[o:o + M] for M, o in zip(MS, off)] for yd in y_dev]
     layers = [fp6.FP6Linear(p_, scales, N_DIM, K_DIM) for p_ in packs]
     h2d = x_host.numel() * 2
-    d2h = y_host.numel() * 2
+    d2h = y_host[0].numel() * 2
     e2e_steps = max(1, args.steps)
+    h2d_stream = torch.cuda.Stream(dev)
+    d2h_stream = torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]     # inputs of buffer b on the device
+    ev_comp = [torch.cuda.Event() for _ in range(2)]   # the step using buffer b has computed
+    ev_out = [torch.cuda.Event() for _ in range(2)]    # buffer b's outputs are on the host
 
     def e2e_step(s):
-        x_dev.copy_(x_host, non_blocking=True)
+        b = s % 2
+        h2d_stream.wait_event(ev_comp[b])            # step s - 2 no longer reads x_dev[b]
+        with torch.cuda.stream(h2d_stream):
+            x_dev[b].copy_(x_host, non_blocking=True)
+        ev_in[b].record(h2d_stream)
+        stream.wait_event(ev_in[b])
+        stream.wait_event(ev_out[b])                 # step s - 2's outputs have left y_dev[b]
         for i in range(len(MS)):
-            layers[(s * len(MS) + i) % copies](x_views[i], out=y_views[i])
-        y_host.copy_(y_dev, non_blocking=True)
+            layers[(s * len(MS) + i) % copies](x_views[b][i], out=y_views[b][i])
+        ev_comp[b].record(stream)
+        d2h_stream.wait_event(ev_comp[b])
+        with torch.cuda.stream(d2h_stream):
+            y_host[b].copy_(y_dev[b], non_blocking=True)
+        ev_out[b].record(d2h_stream)
+
+    def drain():
+        for b in range(2):
+            stream.wait_event(ev_out[b])
 
     with torch.cuda.stream(stream):
         for s in range(args.warmup):
             e2e_step(s)
+        drain()
     torch.cuda.synchronize()
     barrier(world)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         e0.record()
+        h2d_stream.wait_event(e0)
+        d2h_stream.wait_event(e0)
         for s in range(e2e_steps):
             e2e_step(s)
+        drain()                                       # every output copy is inside the region
         e1.record()
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
