@@ -679,12 +679,14 @@ def main():
         args.warmup = 3
     if args.sweep:
         return run_sweep(args)
+    if args.impl == "reference":
+        # The reference arm runs on the host cores of rank 0 alone and uses no
+        # collective: under torchrun the other ranks exit without work, and no
+        # process group (nor CUDA) is set up for it.
+        return run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")))
     world, rank, local = dist_setup(args)
     try:
-        if args.impl == "reference":
-            rc = run_reference(args, world, rank)
-        else:
-            rc = run_fp6(args, world, rank, local)
+        rc = run_fp6(args, world, rank, local)
     finally:
         if world > 1:
             import torch.distributed as dist
