@@ -75,3 +75,31 @@ def test_algorithmic_bytes():
     # packed weights, fp16 scales, fp16 activations of one launch
     assert bench.algo_bytes(1, 8192, 8192) == 0.75 * 8192 * 8192 + 2 * 8192 + 2 * 8192
     assert bench.algo_bytes(16, 8192, 8192, 0.5) == 0.5 * 8192 * 8192 + 2 * 8192 + 2 * 16 * 8192
+
+
+_MAX_CHILD = r"""
+import os, sys, datetime
+sys.path.insert(0, os.environ["REPO"])
+import torch.distributed as dist
+import bench
+dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+rank = dist.get_rank()
+bench.barrier(2)
+t = bench.max_over_ranks(1.5 + rank, 2)          # rank 1 is the slower one
+assert t == 2.5, t
+assert bench.max_over_ranks(7.0, 1) == 7.0       # one rank: no collective
+dist.destroy_process_group()
+open(os.path.join(os.environ["OUT"], f"ok{rank}"), "w").close()
+"""
+
+
+def test_step_time_is_the_max_over_two_ranks(tmp_path):
+    """The timing of an N-rank run is the slowest rank's (gloo ranks on the CPU)."""
+    script = tmp_path / "max_child.py"
+    script.write_text(_MAX_CHILD)
+    env = dict(os.environ, REPO=ROOT, OUT=str(tmp_path))
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(_free_port()), str(script)]
+    out = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr[-2000:]
+    assert (tmp_path / "ok0").exists() and (tmp_path / "ok1").exists()
