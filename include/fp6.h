@@ -126,7 +126,9 @@ size_t fp6_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
  *              bytes (zeroed once before first use, see above); may be NULL
  *              only when that size is 0
  * Concurrent calls must not share a workspace.  Deterministic: the same
- * inputs give the same bits on every run.
+ * inputs give the same bits on every run.  No block of the kernel waits on
+ * another, so the call completes however many of its blocks run at once
+ * (other streams' kernels, an MPS limit or a green context may hold SMs).
  * Launch: programmatic dependent launch.  The kernel may start before the
  * previous kernel in the stream has finished and begins streaming `packed`
  * then; x, scales and every output are touched only after that kernel has
